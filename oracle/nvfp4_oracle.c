@@ -1,0 +1,281 @@
+/*
+ * Oracle for the NVFP4 KV-cache append and block-causal chunk attention path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or
+ * load this file; only the tests, the smoke check and the CPU-baseline leg of
+ * the benchmark do.  It shares no code, header, table or constant generator
+ * with the CUDA library.
+ *
+ * What it follows:
+ *  - "NVlabs/LongLive 2.0: NVFP4 parallel infrastructure for long video
+ *    generation", section "NVFP4, sequence parallel and the async decode path":
+ *    the KV cache is stored in the same 4-bit NVFP4 format as the W4A4
+ *    generator, and the listed optimisations include in-place quantized KV
+ *    updates and FP4 KV dequantization.
+ *  - "NVlabs LongLive" (refft.com), Core Analysis block "How do KV-cache
+ *    relative RoPE and TriAttention work together": positions are assigned
+ *    relative to the cache, so appended chunks do not drift.
+ *  - The workload contract of the tiny reference case (2 heads, head_dim 128,
+ *    8x8 tokens per frame): E2M1 element codes, one E4M3 scale per 16
+ *    contiguous elements, a per-head FP32 global scale equal to the first
+ *    chunk's amax divided by 6*448, round-to-nearest-even everywhere,
+ *    saturation at +-6 and 448, keys cached before RoPE, 3D RoPE split
+ *    44/42/42 over (frame, h, w) with base 10000.
+ *
+ * Precision: the scale arithmetic is FP32 as the contract fixes it (each FP32
+ * operation is evaluated in double and rounded once to float, which is exact
+ * IEEE single rounding for one +,-,*,/ because 53 >= 2*24+2); everything after
+ * dequantization (RoPE, logits, softmax, weighted sum) is fp64.
+ *
+ * Compile with -ffp-contract=off and without -ffast-math.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ---------------------------------------------------------------- FP32 ops */
+
+static float f32_mul(float a, float b) { return (float)((double)a * (double)b); }
+static float f32_div(float a, float b) { return (float)((double)a / (double)b); }
+
+/* ------------------------------------------------------------ E2M1 format */
+
+/* E2M1: bit 3 sign, bits 2..1 exponent (bias 1), bit 0 mantissa.
+ * Exponent 0 is subnormal: value = m * 0.5.  Otherwise 2^(e-1) * (1 + m/2). */
+double oracle_e2m1_decode(uint8_t code)
+{
+    int s = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    double mag = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return s ? -mag : mag;
+}
+
+/* Nearest E2M1 magnitude by exhaustive search over the eight magnitude codes;
+ * a tie goes to the even code (mantissa bit 0).  Magnitudes above 6 saturate
+ * to 6 (stated explicitly: for huge values the fp64 distances to 4 and 6
+ * would compare equal).  A value whose magnitude rounds to zero is stored as
+ * 0x0 (no negative zero). */
+uint8_t oracle_e2m1_encode(float y)
+{
+    double a = fabs((double)y);
+    int best = 0;
+    double best_err = INFINITY;
+    if (a > 6.0) return (uint8_t)(y < 0.0f ? 0xF : 0x7);
+    for (int c = 0; c < 8; ++c) {
+        double err = fabs(oracle_e2m1_decode((uint8_t)c) - a);
+        if (err < best_err || (err == best_err && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_err = err;
+        }
+    }
+    if (best != 0 && y < 0.0f) best |= 8;
+    return (uint8_t)best;
+}
+
+/* ------------------------------------------------------------ E4M3 format */
+
+/* E4M3 ("fn" variant): bit 7 sign, bits 6..3 exponent (bias 7), bits 2..0
+ * mantissa.  Exponent 0 is subnormal: m * 2^-9.  S.1111.111 is NaN, there is
+ * no infinity, the largest finite value is 1.75 * 2^8 = 448. */
+double oracle_e4m3_decode(uint8_t b)
+{
+    int s = (b >> 7) & 1, e = (b >> 3) & 15, m = b & 7;
+    double mag;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) mag = ldexp((double)m, -9);
+    else mag = ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -mag : mag;
+}
+
+/* Nearest non-negative finite E4M3 value by exhaustive search over codes
+ * 0x00..0x7E; a tie goes to the even code.  The caller clamps at 448 first,
+ * as the block-scale rule does. */
+uint8_t oracle_e4m3_encode(float t)
+{
+    double a = (double)t;
+    int best = 0;
+    double best_err = INFINITY;
+    for (int c = 0; c <= 0x7E; ++c) {
+        double err = fabs(oracle_e4m3_decode((uint8_t)c) - a);
+        if (err < best_err || (err == best_err && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_err = err;
+        }
+    }
+    return (uint8_t)best;
+}
+
+/* ---------------------------------------------------------- NVFP4 scales */
+
+/* Per-head global scale: s_g = fl32(amax / (6 * 448)).  A zero amax (or one
+ * so small that s_g would not be a normal float) gives s_g = 1. */
+float oracle_global_scale(float amax)
+{
+    float s = f32_div(amax, 2688.0f);
+    if (!(s >= 1.17549435e-38f)) s = 1.0f;
+    return s;
+}
+
+/* amax over n values (bf16 values carried as float). */
+float oracle_amax(const float *x, int64_t n)
+{
+    float m = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        float a = fabsf(x[i]);
+        if (a > m) m = a;
+    }
+    return m;
+}
+
+/* One 16-element block:
+ *   amax16 = max |x_i|
+ *   t      = fl32(amax16 / fl32(6 * s_g))
+ *   s_b    = 448 if t >= 448, else E4M3_RNE(t)
+ *   y_i    = fl32(x_i / fl32(s_b * s_g)),   q_i = E2M1_RNE_sat(y_i)
+ * s_b = 0 (zero block or scale underflow) gives sixteen zero codes.
+ * Element 2i goes to the low nibble of byte i, element 2i+1 to the high one. */
+void oracle_quantize_block16(const float *x, float s_g, uint8_t *codes8, uint8_t *scale)
+{
+    float amax16 = oracle_amax(x, 16);
+    float t = f32_div(amax16, f32_mul(6.0f, s_g));
+    uint8_t sb = (t >= 448.0f) ? (uint8_t)0x7E : oracle_e4m3_encode(t);
+    float s_b = (float)oracle_e4m3_decode(sb);
+    *scale = sb;
+    memset(codes8, 0, 8);
+    if (s_b == 0.0f) return;
+    float d = f32_mul(s_b, s_g);
+    for (int i = 0; i < 16; ++i) {
+        uint8_t q = oracle_e2m1_encode(f32_div(x[i], d));
+        codes8[i >> 1] |= (uint8_t)(q << ((i & 1) * 4));
+    }
+}
+
+/* Quantize n_rows rows of 128 elements (one token-head each) with one global
+ * scale: codes [n_rows][64], scales [n_rows][8]. */
+void oracle_quantize_rows(const float *x, int64_t n_rows, float s_g, uint8_t *codes, uint8_t *scales)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n_rows; ++r)
+        for (int blk = 0; blk < 8; ++blk)
+            oracle_quantize_block16(x + r * 128 + blk * 16, s_g, codes + r * 64 + blk * 8,
+                                    scales + r * 8 + blk);
+}
+
+/* Dequantize rows: value = e2m1(code) * s_b * s_g, in fp64 (exact). */
+void oracle_dequant_rows(const uint8_t *codes, const uint8_t *scales, int64_t n_rows, float s_g,
+                         double *out)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n_rows; ++r)
+        for (int i = 0; i < 128; ++i) {
+            uint8_t byte = codes[r * 64 + i / 2];
+            uint8_t q = (i & 1) ? (byte >> 4) : (byte & 15);
+            double s_b = oracle_e4m3_decode(scales[r * 8 + i / 16]);
+            out[r * 128 + i] = oracle_e2m1_decode(q) * s_b * (double)s_g;
+        }
+}
+
+/* ------------------------------------------------------------------ RoPE */
+
+/* 3D RoPE on one 128-channel vector, in place, fp64.  Channels are split in
+ * three consecutive segments of widths split[0..2] for the (frame, h, w)
+ * axes.  Inside a segment of width d, pair i is channels (2i, 2i+1) of the
+ * segment, rotated by angle pos * base^(-2i/d):
+ *   (x, y) -> (x cos a - y sin a, x sin a + y cos a). */
+void oracle_rope3d(double *x, const int *pos3, const int *split, double base)
+{
+    int off = 0;
+    for (int ax = 0; ax < 3; ++ax) {
+        int d = split[ax];
+        for (int i = 0; i < d / 2; ++i) {
+            double theta = pow(base, -2.0 * i / (double)d);
+            double a = (double)pos3[ax] * theta;
+            double c = cos(a), s = sin(a);
+            double x0 = x[off + 2 * i], x1 = x[off + 2 * i + 1];
+            x[off + 2 * i] = x0 * c - x1 * s;
+            x[off + 2 * i + 1] = x0 * s + x1 * c;
+        }
+        off += d;
+    }
+}
+
+/* ------------------------------------------------------------- Attention */
+
+/* Chunk attention for one (batch, head), fp64.
+ *   q      [Lq][128]   query values (bf16 inputs as float), before RoPE
+ *   k, v   [Lk][128]   dequantized cached keys (before RoPE) and values
+ *   k_frame_pos [Lk]   RoPE frame index of each key (its order in the cache)
+ *   k_tok  [Lk]        token index of each key inside its frame
+ *   q_frame_pos [Lq]   RoPE frame index of each query row
+ *   q_tok  [Lq]        token index of each query row inside its frame
+ *   rows   [n_rows]    which query rows to compute (all keys are visible to
+ *                      every listed row; masking is done by the caller's
+ *                      choice of keys)
+ *   out    [n_rows][128], lse [n_rows] (natural log of the softmax sum,
+ *                      including the max)
+ * Logits are (R q) . (R k) / sqrt(128); softmax with max subtraction. */
+void oracle_attention_rows(const float *q, const double *k, const double *v, int64_t Lk,
+                           const int *k_frame_pos, const int *k_tok, const int *q_frame_pos,
+                           const int *q_tok, const int64_t *rows, int64_t n_rows, int grid_w,
+                           const int *split, double base, double *out, double *lse)
+{
+    double *kr = (double *)malloc(sizeof(double) * (size_t)Lk * 128);
+    #pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < Lk; ++j) {
+        int pos3[3] = {k_frame_pos[j], k_tok[j] / grid_w, k_tok[j] % grid_w};
+        memcpy(kr + j * 128, k + j * 128, sizeof(double) * 128);
+        oracle_rope3d(kr + j * 128, pos3, split, base);
+    }
+    const double scale = 1.0 / sqrt(128.0);
+    #pragma omp parallel
+    {
+        double *logit = (double *)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+        #pragma omp for schedule(dynamic, 1)
+        for (int64_t ri = 0; ri < n_rows; ++ri) {
+            int64_t r = rows[ri];
+            double qr[128];
+            for (int i = 0; i < 128; ++i) qr[i] = (double)q[r * 128 + i];
+            int pos3[3] = {q_frame_pos[r], q_tok[r] / grid_w, q_tok[r] % grid_w};
+            oracle_rope3d(qr, pos3, split, base);
+            double m = -INFINITY;
+            for (int64_t j = 0; j < Lk; ++j) {
+                double s = 0.0;
+                for (int i = 0; i < 128; ++i) s += qr[i] * kr[j * 128 + i];
+                logit[j] = s * scale;
+                if (logit[j] > m) m = logit[j];
+            }
+            double acc[128];
+            for (int i = 0; i < 128; ++i) acc[i] = 0.0;
+            double l = 0.0;
+            for (int64_t j = 0; j < Lk; ++j) {
+                double p = exp(logit[j] - m);
+                l += p;
+                for (int i = 0; i < 128; ++i) acc[i] += p * v[j * 128 + i];
+            }
+            for (int i = 0; i < 128; ++i) out[ri * 128 + i] = (Lk > 0) ? acc[i] / l : 0.0;
+            if (lse) lse[ri] = (Lk > 0) ? m + log(l) : -INFINITY;
+        }
+        free(logit);
+    }
+    free(kr);
+}
+
+/* ------------------------------------------------------ array entry points */
+
+/* Block-scale code for a scale ratio t (the clamp at 448 included). */
+uint8_t oracle_block_scale_code(float t)
+{
+    return (t >= 448.0f) ? (uint8_t)0x7E : oracle_e4m3_encode(t);
+}
+
+void oracle_e2m1_encode_array(const float *y, int64_t n, uint8_t *out)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_e2m1_encode(y[i]);
+}
+
+void oracle_block_scale_code_array(const float *t, int64_t n, uint8_t *out)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_block_scale_code(t[i]);
+}

@@ -1,0 +1,122 @@
+"""Streaming oracle: the whole AR loop on the CPU (test infrastructure only).
+
+One AR step is append-then-attend (reading: a step quantizes the new chunk's
+K/V with the per-head global scale fixed by step 1, appends it to the sink +
+window ring, then the chunk's queries attend over every visible cached frame,
+their own frames included).  Keys are cached before RoPE and rotated at read
+time, following "NVlabs LongLive" (refft.com), Core Analysis block "How do
+KV-cache relative RoPE and TriAttention work together".
+
+Inputs come from ``kvsynth`` only; no value comes from the CUDA path.
+"""
+from __future__ import annotations
+
+from typing import Dict, List, Optional, Tuple
+
+import numpy as np
+
+import kvsynth
+from . import amax as _amax, attention_rows, dequant_rows, global_scale, quantize_rows
+from .ring import OracleRing
+
+
+class OracleStream:
+    def __init__(self, wl: kvsynth.Workload, seed: int = 0,
+                 shot_sched: Optional[List[List[int]]] = None, keep_inputs: bool = True):
+        self.wl = wl
+        self.seed = seed
+        self.rings = [OracleRing(wl.S, wl.W, wl.C) for _ in range(wl.B)]
+        self.sched = shot_sched if shot_sched is not None else kvsynth.shot_schedule(wl, seed)
+        self.s_g: Optional[np.ndarray] = None      # [2, B, H] float32 (K, V)
+        self.store: Dict[Tuple[int, int], dict] = {}
+        self.step_no = 0
+        self.keep_inputs = keep_inputs
+        self.q = None                              # bf16 Q of the current step
+
+    # ------------------------------------------------------------ append
+
+    def _scales_from(self, k, v) -> np.ndarray:
+        wl = self.wl
+        s = np.zeros((2, wl.B, wl.H), np.float32)
+        for t, x in enumerate((k, v)):
+            xf = x.float().numpy()
+            for b in range(wl.B):
+                for h in range(wl.H):
+                    s[t, b, h] = global_scale(_amax(np.ascontiguousarray(xf[b, :, h, :])))
+        return s
+
+    def step(self, k=None, v=None, q=None):
+        """Advance one AR step; returns {b: [new frame indices]}."""
+        wl = self.wl
+        self.step_no += 1
+        if k is None or v is None or q is None:
+            x = kvsynth.chunk_qkv(wl, self.step_no, self.seed)
+            k, v, q = x["k"], x["v"], x["q"]
+        self.q = q
+        if self.step_no == 1:
+            self.s_g = self._scales_from(k, v)
+        new = {}
+        kf = k.float().numpy()
+        vf = v.float().numpy()
+        for b, ring in enumerate(self.rings):
+            ring.begin_shot(self.sched[b][self.step_no - 1])
+            need = len(ring.frames) + wl.C - ring.capacity
+            if need > 0:
+                for fid in ring.evict(need):
+                    self.store.pop((b, fid), None)
+            fids = ring.append()
+            for c, fid in enumerate(fids):
+                sl = slice(c * wl.T, (c + 1) * wl.T)
+                ent = {}
+                for name, xf, t in (("k", kf, 0), ("v", vf, 1)):
+                    rows = np.ascontiguousarray(xf[b, sl].transpose(1, 0, 2))   # [H, T, D]
+                    codes = np.zeros((wl.H, wl.T, 64), np.uint8)
+                    scales = np.zeros((wl.H, wl.T, 8), np.uint8)
+                    for h in range(wl.H):
+                        codes[h], scales[h] = quantize_rows(rows[h], self.s_g[t, b, h])
+                    ent[name + "_codes"] = codes
+                    ent[name + "_scales"] = scales
+                    if self.keep_inputs:
+                        ent[name + "_bf16"] = rows
+                self.store[(b, fid)] = ent
+            new[b] = fids
+        return new
+
+    # ------------------------------------------------------------- read
+
+    def frame(self, b: int, fid: int) -> dict:
+        return self.store[(b, fid)]
+
+    def visible_kv(self, b: int, h: int, quantized: bool = True):
+        """Visible keys/values of the newest chunk for (b, h) in logical order.
+
+        Returns (k [Lk,128] f64, v [Lk,128] f64, k_frame_pos [Lk], k_tok [Lk]).
+        ``quantized=False`` gives the bf16 cache (the bf16-KV twin)."""
+        wl = self.wl
+        ks, vs, fpos, tok = [], [], [], []
+        for fid, rank in self.rings[b].visible():
+            e = self.store[(b, fid)]
+            if quantized:
+                ks.append(dequant_rows(e["k_codes"][h], e["k_scales"][h], self.s_g[0, b, h]))
+                vs.append(dequant_rows(e["v_codes"][h], e["v_scales"][h], self.s_g[1, b, h]))
+            else:
+                ks.append(e["k_bf16"][h].astype(np.float64))
+                vs.append(e["v_bf16"][h].astype(np.float64))
+            fpos.append(np.full(wl.T, rank, np.int32))
+            tok.append(np.arange(wl.T, dtype=np.int32))
+        if not ks:
+            z = np.zeros((0, 128))
+            return z, z, np.zeros(0, np.int32), np.zeros(0, np.int32)
+        return np.concatenate(ks), np.concatenate(vs), np.concatenate(fpos), np.concatenate(tok)
+
+    def query_positions(self, b: int):
+        wl = self.wl
+        l = np.arange(wl.Lq)
+        return (self.rings[b].query_pos0() + l // wl.T).astype(np.int32), (l % wl.T).astype(np.int32)
+
+    def attention(self, b: int, h: int, rows, quantized: bool = True):
+        """Oracle outputs (fp64) for query rows ``rows`` of (b, h) at the current step."""
+        k, v, fpos, tok = self.visible_kv(b, h, quantized)
+        qpos, qtok = self.query_positions(b)
+        q = self.q[b, :, h, :]
+        return attention_rows(q, k, v, fpos, tok, qpos, qtok, rows, self.wl.grid_w)
