@@ -1,0 +1,390 @@
+"""Benchmark of the NVFP4 KV-cache hot path on B200.
+
+One step = one AR step of the 1.3B-like streaming workload (batch 1, 12 heads,
+head_dim 128, 1560 tokens per frame, chunk 3 frames = 4680 query tokens,
+sink 3 + window 18 frames = 32760 keys per query) in steady state:
+kv_ring_evict + nvfp4_kv_append + chunk_attention_nvfp4kv.  Inputs are seeded
+synthetic bf16 N(0,1) with 1% K outlier channels x8.  Four independent caches
+(one per emulated layer) and four input sets are cycled, so each step reads
+a cache and inputs that are not L2-resident (4 x ~100 MB > 126 MB L2).
+
+Prints one JSON line (rank 0).  --impl reference times the CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4-KV chunk attention TFLOP/s & query tok/s; KV quant-append GB/s"
+N_LAYERS = 4
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def workload_numbers(wl):
+    """Algorithmic work per step (see the per-kernel accounting in the docs)."""
+    T, Lq = wl.T, wl.Lq
+    n_keys = (wl.S + wl.W) * T
+    flop = 4.0 * wl.B * wl.H * Lq * n_keys * 128
+    # append: read bf16 K and V, write codes (64 B) + scales (8 B) per token-head
+    append_bytes = wl.B * Lq * wl.H * (2 * 256 + 2 * 72)
+    twin_append_bytes = wl.B * Lq * wl.H * (2 * 256 + 2 * 256)
+    # attention HBM bytes: Q in, O out, every visible K/V row once
+    attn_bytes = wl.B * wl.H * (2 * Lq * 256 + n_keys * 2 * 72)
+    return dict(flop=flop, append_bytes=append_bytes, twin_append_bytes=twin_append_bytes,
+                attn_bytes=attn_bytes, n_keys=n_keys)
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def _dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# --------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import kvsynth
+    import nvfp4_kv_cache_append_b200 as nv
+
+    ws, rank, local = _dist_env()
+    torch.cuda.set_device(local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    wl = kvsynth.WORKLOADS[args.workload]
+    num = workload_numbers(wl)
+    fp4 = args.kv == "nvfp4"
+    kvd = nv.NVKV_KV_NVFP4 if fp4 else nv.NVKV_KV_BF16
+    stream = torch.cuda.Stream()
+    torch.cuda.set_stream(stream)
+
+    # inputs: N_LAYERS seeded sets, resident in HBM before timing
+    sets = []
+    for i in range(N_LAYERS):
+        x = kvsynth.chunk_qkv(wl, 1000 + i, seed=rank)
+        sets.append({k: v.cuda() for k, v in x.items()})
+    caches = [nv.KVCache(wl.B, wl.H, wl.grid_h, wl.grid_w, wl.C, wl.S, wl.W, kvd)
+              for _ in range(N_LAYERS)]
+    outs = [torch.empty_like(sets[0]["q"]) for _ in range(N_LAYERS)]
+    # fill every ring to steady state (window full)
+    fill = (wl.S + wl.W) // wl.C
+    for c in caches:
+        for s in range(fill):
+            x = sets[s % N_LAYERS]
+            c.step(x["q"], x["k"], x["v"], out=outs[0])
+    torch.cuda.synchronize()
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def one_step(i, timing):
+        li = i % N_LAYERS
+        c, x = caches[li], sets[(i + 1) % N_LAYERS]
+        need = wl.C - c.free_frames(0)
+        e0 = e1 = e2 = None
+        if timing:
+            e0 = ev(); e0.record(stream)
+        if need > 0:
+            c.evict(need)
+        c.append(x["k"], x["v"], stream=stream)
+        if timing:
+            e1 = ev(); e1.record(stream)
+        c.attention(x["q"], out=outs[li], stream=stream)
+        if timing:
+            e2 = ev(); e2.record(stream)
+        return e0, e1, e2
+
+    for i in range(args.warmup):
+        one_step(i, False)
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    t_start, t_end = ev(), ev()
+    t_start.record(stream)
+    marks = [one_step(args.warmup + i, True) for i in range(args.steps)]
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    app_ms = [a.elapsed_time(b) for a, b, _ in marks]
+    att_ms = [b.elapsed_time(c) for _, b, c in marks]
+    if ws > 1:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    for c in caches:
+        assert c.device_status() == 0, "device-side pipeline error"
+
+    # end to end through the same calls with host buffers: pinned H2D of the
+    # step's q/k/v, the step, D2H of the output
+    host = [{k: v.cpu().pin_memory() for k, v in s.items()} for s in sets]
+    host_out = torch.empty(sets[0]["q"].shape, dtype=torch.bfloat16).pin_memory()
+    dev_in = {k: torch.empty_like(v) for k, v in sets[0].items()}
+    h2d = sum(v.numel() * v.element_size() for v in host[0].values())
+    d2h = host_out.numel() * host_out.element_size()
+
+    def e2e_step(i):
+        li = i % N_LAYERS
+        for k, v in host[(i + 1) % N_LAYERS].items():
+            dev_in[k].copy_(v, non_blocking=True)
+        c = caches[li]
+        need = wl.C - c.free_frames(0)
+        if need > 0:
+            c.evict(need)
+        c.append(dev_in["k"], dev_in["v"], stream=stream)
+        c.attention(dev_in["q"], out=outs[li], stream=stream)
+        host_out.copy_(outs[li], non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    a, b = ev(), ev()
+    a.record(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b)
+    if ws > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    peaks = _peaks()
+    K = args.steps
+    ms_step = total_ms / K
+    tok_per_step = wl.B * wl.Lq
+    value = ws * tok_per_step * K / (total_ms / 1e3)
+    att_avg = sum(att_ms) / K
+    app_avg = sum(app_ms) / K
+    attn_tflops = num["flop"] / (att_avg / 1e3) / 1e12
+    app_bytes = num["append_bytes"] if fp4 else num["twin_append_bytes"]
+    append_gbs = app_bytes / (app_avg / 1e3) / 1e9
+    peak = peaks["bf16_tflops_sustained"] if K * ms_step > 2000 else peaks["bf16_tflops"]
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "query tok/s",
+        "n_gpus": ws,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e2m1/e4m3 cache, f16 MMA, f32 accumulate" if fp4 else "bf16 MMA, f32 accumulate",
+        "data": "synthetic (seeded bf16 N(0,1), 1% K outlier channels x8)",
+        "config": {"workload": f"{wl.name}: B{wl.B} H{wl.H} D128 T{wl.T} ({wl.grid_h}x{wl.grid_w}) "
+                               f"C{wl.C} S{wl.S} W{wl.W}, {wl.Lq} query tokens, {num['n_keys']} keys",
+                   "kv_cache": args.kv, "layers_cycled": N_LAYERS,
+                   "l2": "inputs and caches larger than L2 (4 independent layers cycled)",
+                   "parallelism": f"replicas x{ws}"},
+        "attn_tflops": attn_tflops,
+        "attn_ms": att_avg,
+        "append_gbs": append_gbs,
+        "append_ms": app_avg,
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak,
+                     "unit": "TFLOP/s", "frac": attn_tflops / peak, "traffic": None,
+                     "kernel": "k_chunk_attn", "peak_source": peaks["source"] + " bf16 (f16 same nominal rate)"},
+        "append_roofline": {"bound": "hbm", "achieved": append_gbs, "peak": peaks["hbm_gbs"],
+                            "unit": "GB/s", "frac": append_gbs / peaks["hbm_gbs"]},
+        "e2e": {"value": ws * tok_per_step * K / (e2e_ms / 1e3), "unit": "query tok/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * K,
+        "clocks": clk,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, seconds=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------ oracle arm
+
+def _oracle_sample(wl, n_rows, seed=0):
+    """Time the oracle on a bounded sample of one steady-state step."""
+    import numpy as np
+
+    import kvsynth
+    import oracle
+
+    x = kvsynth.chunk_qkv(wl, 1, seed)
+    kf, vf = x["k"].float().numpy(), x["v"].float().numpy()
+    t0 = time.perf_counter()
+    # quantize-append of the whole chunk (K and V, every head)
+    for arr in (kf, vf):
+        for h in range(wl.H):
+            rows = np.ascontiguousarray(arr[0, :, h])
+            oracle.quantize_rows(rows, oracle.global_scale(oracle.amax(rows)))
+    t_app = time.perf_counter() - t0
+    # attention of n_rows query tokens (all heads) over 32760 keys
+    n_keys = (wl.S + wl.W) * wl.T
+    rng = np.random.default_rng(seed)
+    k = rng.standard_normal((n_keys, 128))
+    v = rng.standard_normal((n_keys, 128))
+    fpos = np.repeat(np.arange(wl.S + wl.W, dtype=np.int32), wl.T)
+    tok = np.tile(np.arange(wl.T, dtype=np.int32), wl.S + wl.W)
+    q = x["q"][0]
+    l = np.arange(wl.Lq)
+    qpos = (wl.S + wl.W - wl.C + l // wl.T).astype(np.int32)
+    qtok = (l % wl.T).astype(np.int32)
+    rows = rng.choice(wl.Lq, n_rows, replace=False)
+    t0 = time.perf_counter()
+    for h in range(wl.H):
+        oracle.attention_rows(q[:, h], k, v, fpos, tok, qpos, qtok, rows, wl.grid_w)
+    t_att = time.perf_counter() - t0
+    per_tok = t_app / wl.Lq + t_att / n_rows
+    return 1.0 / per_tok, t_app, t_att
+
+
+def cpu_baseline(wl, seconds=20.0):
+    import oracle
+    oracle.build()
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    n_rows = max(8, int(seconds * 6))
+    value, t_app, t_att = _oracle_sample(wl, n_rows)
+    return {"value": value, "unit": "query tok/s", "cores": cores, "kind": "oracle",
+            "sample": f"one {wl.name} step: full-chunk quantize ({wl.Lq} tokens x {wl.H} heads, "
+                      f"K and V) + attention of {n_rows} query tokens x {wl.H} heads over "
+                      f"{(wl.S + wl.W) * wl.T} keys; tok/s = 1 / (append s/token + attention s/token)",
+            "append_s": t_app, "attention_s": t_att}
+
+
+def run_reference(args):
+    import kvsynth
+    ws, rank, _ = _dist_env()
+    if rank != 0:
+        return
+    wl = kvsynth.WORKLOADS[args.workload]
+    import oracle
+    oracle.build()
+    n_rows = 8
+    for _ in range(args.warmup):
+        _oracle_sample(wl, 2)
+    vals = []
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        v, _, _ = _oracle_sample(wl, n_rows, seed=i)
+        vals.append(v)
+    wall = time.perf_counter() - t0
+    value = len(vals) / sum(1.0 / v for v in vals)
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    sample = (f"per step: full-chunk quantize + attention of {n_rows} query tokens x {wl.H} heads "
+              f"over {(wl.S + wl.W) * wl.T} keys")
+    line = {"metric": METRIC, "value": value, "unit": "query tok/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * wall / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded bf16 N(0,1), 1% K outlier channels x8)",
+            "config": {"workload": f"{wl.name}", "parallelism": "host cores"},
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "query tok/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "query tok/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="stream1p3b")
+    ap.add_argument("--kv", default="nvfp4", choices=["nvfp4", "bf16"])
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,255 @@
+/*
+ * nvkv.h -- C ABI of the NVFP4 KV-cache append and block-causal chunk
+ * attention library for B200 (sm_100a).
+ *
+ * The path it implements, per autoregressive (AR) step of a streaming video
+ * diffusion generator:
+ *
+ *   kv_ring_evict            drop the oldest non-sink frames when the ring is full
+ *   nvfp4_kv_append          quantize the new chunk's K/V to NVFP4 and write it,
+ *                            in place, into free frame slots of the cache
+ *   chunk_attention_nvfp4kv  the chunk's queries attend over the dequantized,
+ *                            RoPE-rotated sink + window K/V
+ *
+ * plus a bf16-KV twin of the cache (bf16_kv_append, chunk_attention_bf16kv).
+ *
+ * Sources: "NVlabs/LongLive 2.0: NVFP4 parallel infrastructure for long video
+ * generation" (hysenlabs.com), section "NVFP4, sequence parallel and the async
+ * decode path": the KV cache is kept in the same NVFP4 format as the W4A4
+ * generator, beside a BF16 path; the listed optimisations are in-place
+ * quantized KV-cache updates, faster FP4 KV dequantization, fused RoPE and
+ * reduced KV-cache synchronisation; attention sinks keep the streaming
+ * generator from drifting and extend to multi-shot video.  "NVlabs LongLive"
+ * (refft.com), Core Analysis block "How do KV-cache relative RoPE and
+ * TriAttention work together": RoPE is applied relative to the cache, so new
+ * chunks append without position drift.  "LongLive: NVIDIA long video
+ * generation" (evermx.com), heading "Multi-Shot Generation": shots attend to
+ * relevant past context without bleeding across cuts.
+ *
+ * NVFP4 format used by the cache (the workload contract of the tiny reference
+ * case): per 16 contiguous head_dim elements one E4M3 block scale
+ *   s_b = E4M3_RNE(min(fl32(amax16 / fl32(6 * s_g)), 448)),
+ * E2M1 codes q = E2M1_RNE_sat(fl32(x / fl32(s_b * s_g))) (a magnitude that
+ * rounds to zero is stored as code 0; s_b = 0 gives all-zero codes), two codes
+ * per byte with element 2i in the low nibble, and one FP32 global scale per
+ * (K or V, batch, head) fixed by the first chunk: s_g = fl32(amax / 2688)
+ * (1 when that is zero or not a normal float).  Dequantized value:
+ * e2m1(q) * s_b * s_g.
+ *
+ * Conventions
+ *  - All device memory is allocated by the caller, once, with the sizes
+ *    nvkv_plane_bytes() and nvkv_attention_workspace_bytes() report.  The
+ *    library never allocates, frees or synchronises; every device call is
+ *    asynchronous and ordered on the stream it is given.
+ *  - Host validation errors are returned before anything is launched and leave
+ *    the ring unchanged.  A launch failure returns NVKV_ERR_CUDA.  Errors found
+ *    on the device (a pipeline wait that ran out of its bound) are written to
+ *    cache->status as an nvkv_status value; the caller reads it after a sync.
+ *  - q, k, v and out are contiguous bf16 tensors [B][Lq][H][128] with
+ *    Lq = C * T tokens (C frames of T = grid_h * grid_w tokens, token t of a
+ *    frame at row t / grid_w, column t % grid_w).  Device pointers must be
+ *    16-byte aligned.
+ *  - The ring (nvkv_ring) is a host-side value owned by the caller.  Kernels
+ *    receive a snapshot of it as a launch parameter: no host-to-device copy and
+ *    no host sync per step.
+ */
+#ifndef NVKV_H
+#define NVKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define NVKV_API __attribute__((visibility("default")))
+#else
+#define NVKV_API
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *nvkv_stream;
+
+typedef enum {
+    NVKV_OK = 0,
+    NVKV_ERR_INVALID_ARG = 1,  /* null pointer, bad size, bad shot id          */
+    NVKV_ERR_UNSUPPORTED = 2,  /* head_dim != 128, limits exceeded, no sm_100  */
+    NVKV_ERR_ALIGNMENT = 3,    /* a device pointer is not 16-byte aligned      */
+    NVKV_ERR_CAPACITY = 4,     /* no room for the chunk (evict first) or too
+                                  few evictable frames; workspace too small    */
+    NVKV_ERR_STATE = 5,        /* bad magic/version, ring does not match desc,
+                                  attention before any append, wrong kv dtype  */
+    NVKV_ERR_CUDA = 6,         /* a CUDA launch failed                         */
+    NVKV_ERR_TIMEOUT = 7       /* device status only: a bounded wait expired   */
+} nvkv_status;
+
+#define NVKV_MAGIC 0x4E564B56u /* "NVKV" */
+#define NVKV_VERSION 1u
+#define NVKV_HEAD_DIM 128
+#define NVKV_MAX_BATCH 16
+#define NVKV_MAX_FRAMES 64     /* S + W */
+#define NVKV_MAX_CHUNK 16      /* C */
+
+enum { NVKV_KV_NVFP4 = 0, NVKV_KV_BF16 = 1 };
+
+/* Problem description (a value type; fill it with nvkv_desc_init). */
+typedef struct {
+    uint32_t magic, version;
+    int32_t B;            /* batch (independent streams)                       */
+    int32_t H;            /* heads                                             */
+    int32_t D;            /* head_dim, must be 128                             */
+    int32_t grid_h;       /* latent rows per frame                             */
+    int32_t grid_w;       /* latent columns per frame; T = grid_h * grid_w      */
+    int32_t C;            /* frames per chunk (per AR step)                    */
+    int32_t S;            /* sink frames (the first S frames ever appended)     */
+    int32_t W;            /* window frames, the current chunk included          */
+    int32_t kv_dtype;     /* NVKV_KV_NVFP4 or NVKV_KV_BF16                      */
+    float rope_base;      /* 10000                                             */
+    int32_t rope_split[3];/* head_dim channels for (frame, h, w): 44, 42, 42    */
+} nvkv_desc;
+
+/* Device planes of one cache (caller-owned; sizes from nvkv_plane_bytes).
+ * R = (S + W) * T rows per (batch, head); physical frame slot p holds rows
+ * [p*T, (p+1)*T).
+ *   NVFP4: k_data/v_data = codes [B][H][R][64] u8, k_scales/v_scales = E4M3
+ *          block scales [B][H][R][8] u8, amax [2][B][H] (float bits, K then
+ *          V), s_g [2][B][H] f32.
+ *   BF16:  k_data/v_data = [B][H][R][128] bf16; the other planes may be NULL.
+ * status: one int32, cleared by the caller; device errors are written here. */
+typedef struct {
+    void *k_data, *v_data;
+    void *k_scales, *v_scales;
+    uint32_t *amax;
+    float *s_g;
+    int32_t *status;
+} nvkv_cache;
+
+enum {
+    NVKV_PLANE_K_DATA = 0, NVKV_PLANE_V_DATA = 1, NVKV_PLANE_K_SCALES = 2,
+    NVKV_PLANE_V_SCALES = 3, NVKV_PLANE_AMAX = 4, NVKV_PLANE_SCALE_G = 5,
+    NVKV_PLANE_STATUS = 6
+};
+
+/* Frame flags in the ring. */
+#define NVKV_FRAME_SINK 1u       /* global attention sink, never evicted        */
+#define NVKV_FRAME_PINNED 2u     /* per-shot sink of the running shot           */
+#define NVKV_FRAME_SHOT_LAST 4u  /* last frame of a shot that has ended          */
+
+/* Ring state of one stream.  Resident frames in logical order: sink frames
+ * first, then the others by age.  The RoPE frame index of a resident frame is
+ * its position in this order. */
+typedef struct {
+    int32_t n_resident;
+    int32_t shot;                         /* running shot id                  */
+    int32_t pin_next;                     /* next chunk is a per-shot sink    */
+    int32_t n_appended;                   /* frames appended so far           */
+    int32_t slot[NVKV_MAX_FRAMES];        /* logical index -> physical slot   */
+    int32_t frame[NVKV_MAX_FRAMES];       /* logical index -> frame number    */
+    int32_t frame_shot[NVKV_MAX_FRAMES];  /* logical index -> shot id         */
+    uint32_t flags[NVKV_MAX_FRAMES];      /* NVKV_FRAME_*                     */
+} nvkv_ring_stream;
+
+typedef struct {
+    uint32_t magic, version;
+    int32_t B, capacity, C, S;            /* copied from the desc at init      */
+    int32_t scales_fixed;                 /* 1 once step 1 fixed the s_g       */
+    int32_t steps;                        /* appends so far                   */
+    nvkv_ring_stream s[NVKV_MAX_BATCH];
+} nvkv_ring;
+
+/* Fill a desc with D = 128, RoPE split 44/42/42 and base 10000.  Returns
+ * NVKV_ERR_INVALID_ARG / NVKV_ERR_UNSUPPORTED for shapes outside the limits
+ * (B <= 16, S + W <= 64, 1 <= C <= min(W, 16), T >= 1, grid_h, grid_w < 65536). */
+NVKV_API nvkv_status nvkv_desc_init(nvkv_desc *desc, int B, int H, int grid_h, int grid_w, int C, int S,
+                           int W, int kv_dtype);
+
+/* Bytes the caller must allocate for one plane (NVKV_PLANE_*) of a cache of
+ * this desc; 0 for planes the dtype does not use or for an invalid desc. */
+NVKV_API size_t nvkv_plane_bytes(const nvkv_desc *desc, int plane);
+
+/* Empty ring for this desc (all frames free, shot 0). */
+NVKV_API nvkv_status nvkv_ring_init(const nvkv_desc *desc, nvkv_ring *ring);
+
+/* Host only, no device work: in every stream, drop the n_frames oldest
+ * resident frames that are neither sink nor pinned (the sink + rolling window
+ * rule: "eviction drops the oldest non-sink frame").  NVKV_ERR_CAPACITY, and
+ * no change, if any stream has fewer evictable frames. */
+NVKV_API nvkv_status kv_ring_evict(const nvkv_desc *desc, nvkv_ring *ring, int n_frames);
+
+/* Host only: stream b starts shot shot_id (>= the running one; equal is a
+ * no-op).  The newest resident frame is marked as its shot's last frame,
+ * every pinned frame is unpinned, and the next chunk appended to b becomes the
+ * new shot's per-shot sink (pinned until the following shot begins).  A chunk
+ * of shot s sees the global sink, all frames of shot s and the last frame of
+ * each earlier shot ("LongLive: NVIDIA long video generation", heading
+ * "Multi-Shot Generation"). */
+NVKV_API nvkv_status kv_ring_begin_shot(const nvkv_desc *desc, nvkv_ring *ring, int b, int shot_id);
+
+/* Host query of what the newest chunk of stream b sees: for each visible frame
+ * in logical order its physical slot, RoPE frame index and frame number
+ * (arrays of at least NVKV_MAX_FRAMES entries, any may be NULL).  Returns the
+ * number of visible frames, or -1 on a bad argument.  *query_pos0 (may be
+ * NULL) receives the RoPE frame index of the newest chunk's first frame. */
+NVKV_API int nvkv_ring_visible(const nvkv_desc *desc, const nvkv_ring *ring, int b, int32_t *slots,
+                      int32_t *rope_pos, int32_t *frames, int32_t *query_pos0);
+
+/* Host only: the ring update of one append without any device work.  Assigns
+ * C free physical slots per stream (lowest free first), records the chunk's
+ * frames as resident (sink flag for the first S frames ever appended, pinned
+ * if the chunk opens a shot) and writes the slots to slots_out[b * C + c]
+ * (may be NULL).  For callers that write a chunk's K/V into those slots with
+ * their own kernel.  NVKV_ERR_CAPACITY (no change) if a stream has fewer than
+ * C free frames. */
+NVKV_API nvkv_status nvkv_ring_push_chunk(const nvkv_desc *desc, nvkv_ring *ring,
+                                          int32_t *slots_out);
+
+/* Quantize-append, in place.  k, v: device bf16 [B][Lq][H][128].  Assigns C
+ * free physical slots per stream (lowest free first), quantizes K and V to
+ * NVFP4 and writes codes and scales into those slots; on the first append it
+ * also measures the per-(K/V, batch, head) amax of the chunk and fixes s_g.
+ * NVKV_ERR_CAPACITY (no change) if a stream has fewer than C free frames. */
+NVKV_API nvkv_status nvfp4_kv_append(const nvkv_desc *desc, const nvkv_cache *cache, nvkv_ring *ring,
+                            const void *k, const void *v, nvkv_stream stream);
+
+/* The bf16-KV twin: same slot logic, the chunk's bf16 K/V copied as is. */
+NVKV_API nvkv_status bf16_kv_append(const nvkv_desc *desc, const nvkv_cache *cache, nvkv_ring *ring,
+                           const void *k, const void *v, nvkv_stream stream);
+
+/* Device workspace the attention calls need (may be 0). */
+NVKV_API size_t nvkv_attention_workspace_bytes(const nvkv_desc *desc);
+
+/* Block-causal chunk attention of the newest chunk.  q: device bf16
+ * [B][Lq][H][128] before RoPE; out: device bf16 [B][Lq][H][128]; lse: NULL or
+ * device f32 [B][H][Lq] (natural-log softmax normaliser, max included).
+ * Every query of the chunk sees every token of every visible frame (its own
+ * chunk included, in full).  Keys are read from the cache, dequantized and
+ * rotated by 3D RoPE at (their frame's RoPE index, h, w); queries are rotated
+ * at (the RoPE index of their own frame, h, w).  Logits use 1/sqrt(128).
+ * NVKV_ERR_STATE if nothing was appended yet. */
+NVKV_API nvkv_status chunk_attention_nvfp4kv(const nvkv_desc *desc, const nvkv_cache *cache,
+                                    const nvkv_ring *ring, const void *q, void *out, float *lse,
+                                    void *workspace, size_t workspace_bytes, nvkv_stream stream);
+
+/* The bf16-KV twin of chunk_attention_nvfp4kv. */
+NVKV_API nvkv_status chunk_attention_bf16kv(const nvkv_desc *desc, const nvkv_cache *cache,
+                                   const nvkv_ring *ring, const void *q, void *out, float *lse,
+                                   void *workspace, size_t workspace_bytes, nvkv_stream stream);
+
+/* Diagnostics: the device conversions the append kernel uses, one value per
+ * element.  y, t: device f32 [n]; codes: device u8 [n].
+ * nvkv_encode_e2m1: E2M1_RNE_sat(y) with negative zero stored as 0.
+ * nvkv_encode_block_scale: E4M3_RNE(min(t, 448)) for t >= 0. */
+NVKV_API nvkv_status nvkv_encode_e2m1(const float *y, uint8_t *codes, size_t n, nvkv_stream stream);
+NVKV_API nvkv_status nvkv_encode_block_scale(const float *t, uint8_t *codes, size_t n, nvkv_stream stream);
+
+NVKV_API const char *nvkv_status_string(nvkv_status status);
+
+/* NVKV_VERSION of the loaded library. */
+NVKV_API uint32_t nvkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVKV_H */

@@ -1,0 +1,139 @@
+"""Caller-side plumbing around the C ABI: device planes allocated once with
+PyTorch (sizes from ``nvkv_plane_bytes``), the host ring, and one method per
+entry point.  PyTorch provides memory and streams only; every step of the
+path runs in libnvkv.so's kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from . import _lib as L
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class KVCache:
+    """One sink + rolling-window KV ring (NVFP4 or bf16) on one CUDA device."""
+
+    def __init__(self, B: int, H: int, grid_h: int, grid_w: int, C: int, S: int, W: int,
+                 kv_dtype: int = L.NVKV_KV_NVFP4, device="cuda"):
+        self.desc = L.nvkv_desc_init(B, H, grid_h, grid_w, C, S, W, kv_dtype)
+        self.ring = L.nvkv_ring_init(self.desc)
+        self.device = torch.device(device)
+        if self.device.type != "cuda":
+            raise ValueError("the cache lives in CUDA device memory")
+        nb = lambda p: L.nvkv_plane_bytes(self.desc, p)
+        alloc = lambda n: torch.zeros(max(n, 16), dtype=torch.uint8, device=self.device)
+        self.k_data = alloc(nb(L.NVKV_PLANE_K_DATA))
+        self.v_data = alloc(nb(L.NVKV_PLANE_V_DATA))
+        fp4 = kv_dtype == L.NVKV_KV_NVFP4
+        self.k_scales = alloc(nb(L.NVKV_PLANE_K_SCALES)) if fp4 else None
+        self.v_scales = alloc(nb(L.NVKV_PLANE_V_SCALES)) if fp4 else None
+        self.amax = alloc(nb(L.NVKV_PLANE_AMAX)) if fp4 else None
+        self.s_g = alloc(nb(L.NVKV_PLANE_SCALE_G)) if fp4 else None
+        self.status = alloc(nb(L.NVKV_PLANE_STATUS))
+        ws = L.nvkv_attention_workspace_bytes(self.desc)
+        self.workspace = alloc(ws) if ws else None
+        self.ws_bytes = ws
+        self.cache = L.nvkv_cache(
+            _ptr(self.k_data).value, _ptr(self.v_data).value,
+            None if self.k_scales is None else self.k_scales.data_ptr(),
+            None if self.v_scales is None else self.v_scales.data_ptr(),
+            None if self.amax is None else self.amax.data_ptr(),
+            None if self.s_g is None else self.s_g.data_ptr(),
+            self.status.data_ptr())
+        self.fp4 = fp4
+
+    # ---------------------------------------------------------------- shape
+    @property
+    def T(self) -> int:
+        return self.desc.grid_h * self.desc.grid_w
+
+    @property
+    def Lq(self) -> int:
+        return self.desc.C * self.T
+
+    @property
+    def rows(self) -> int:
+        return (self.desc.S + self.desc.W) * self.T
+
+    def footprint_bytes(self) -> int:
+        ts = [self.k_data, self.v_data, self.k_scales, self.v_scales, self.amax, self.s_g,
+              self.status, self.workspace]
+        return sum(t.numel() * t.element_size() for t in ts if t is not None)
+
+    # ---------------------------------------------------------------- views
+    def codes(self, which: str) -> torch.Tensor:
+        """[B, H, R, 64] u8 codes (NVFP4) or [B, H, R, 128] bf16 (twin)."""
+        t = self.k_data if which == "k" else self.v_data
+        d = self.desc
+        if self.fp4:
+            return t[: d.B * d.H * self.rows * 64].view(d.B, d.H, self.rows, 64)
+        return t.view(torch.bfloat16)[: d.B * d.H * self.rows * 128].view(d.B, d.H, self.rows, 128)
+
+    def scales(self, which: str) -> torch.Tensor:
+        t = self.k_scales if which == "k" else self.v_scales
+        d = self.desc
+        return t[: d.B * d.H * self.rows * 8].view(d.B, d.H, self.rows, 8)
+
+    def global_scales(self) -> torch.Tensor:
+        return self.s_g.view(torch.float32)[: 2 * self.desc.B * self.desc.H].view(
+            2, self.desc.B, self.desc.H)
+
+    def device_status(self) -> int:
+        return int(self.status.view(torch.int32)[0].item())
+
+    # -------------------------------------------------------------- entries
+    def evict(self, n_frames: int) -> None:
+        L.kv_ring_evict(self.desc, self.ring, n_frames)
+
+    def begin_shot(self, b: int, shot_id: int) -> None:
+        L.kv_ring_begin_shot(self.desc, self.ring, b, shot_id)
+
+    def visible(self, b: int):
+        return L.nvkv_ring_visible(self.desc, self.ring, b)
+
+    def free_frames(self, b: int = 0) -> int:
+        return self.desc.S + self.desc.W - self.ring.s[b].n_resident
+
+    def append(self, k: torch.Tensor, v: torch.Tensor, stream=None) -> None:
+        self._check_io(k)
+        self._check_io(v)
+        fn = L.nvfp4_kv_append if self.fp4 else L.bf16_kv_append
+        fn(self.desc, self.cache, self.ring, _ptr(k), _ptr(v), _stream(stream))
+
+    def attention(self, q: torch.Tensor, out: Optional[torch.Tensor] = None,
+                  lse: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        self._check_io(q)
+        if out is None:
+            out = torch.empty_like(q)
+        self._check_io(out)
+        fn = L.chunk_attention_nvfp4kv if self.fp4 else L.chunk_attention_bf16kv
+        fn(self.desc, self.cache, self.ring, _ptr(q), _ptr(out), _ptr(lse), _ptr(self.workspace),
+           self.ws_bytes, _stream(stream))
+        return out
+
+    def step(self, q, k, v, out=None, lse=None, stream=None) -> torch.Tensor:
+        """One AR step: evict when full, quantize-append, attend."""
+        need = self.desc.C - min(self.free_frames(b) for b in range(self.desc.B))
+        if need > 0:
+            self.evict(need)
+        self.append(k, v, stream)
+        return self.attention(q, out, lse, stream)
+
+    def _check_io(self, t: torch.Tensor) -> None:
+        d = self.desc
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(
+                t.shape) != (d.B, self.Lq, d.H, 128):
+            raise ValueError(f"expected contiguous CUDA bf16 [{d.B}, {self.Lq}, {d.H}, 128], got "
+                             f"{t.dtype} {tuple(t.shape)} on {t.device}")

@@ -1,0 +1,260 @@
+// NVFP4 quantize-append and bf16 append kernels (sm_100a).
+//
+// In-place quantized KV-cache update ("NVlabs/LongLive 2.0: NVFP4 parallel
+// infrastructure for long video generation", section "NVFP4, sequence
+// parallel and the async decode path").  Format: E2M1 codes, one E4M3 scale
+// per 16 head_dim elements, one FP32 global scale per (K/V, batch, head):
+//   s_g  = fl32(amax(first chunk) / 2688)        (1 if not a normal float)
+//   s_b  = E4M3_RNE(min(fl32(amax16 / fl32(6 s_g)), 448))
+//   q_i  = E2M1_RNE_sat(fl32(x_i / fl32(s_b s_g)))   (s_b = 0 -> all zero)
+// Element 2i is the low nibble of byte i; a magnitude that rounds to zero is
+// stored as code 0.  The FP32 operations are IEEE round-to-nearest (no
+// contraction, true division), so the codes are bit-exact.
+//
+// Memory: HBM-bound.  Each thread owns one 16-element block: two 16-byte
+// loads of bf16 input (a warp reads 1 KB contiguous), one 8-byte code store
+// and one scale byte (eight threads of a token-head write 64 contiguous code
+// bytes).  Rows go straight into the physical frame slot (no staging).
+#include <cuda_bf16.h>
+
+#include "nvkv_internal.h"
+
+namespace nvkv {
+namespace {
+
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p)
+{
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// max |x| over the eight bf16 values of two words pairs, as a float.
+__device__ __forceinline__ uint32_t absmax_bits(uint4 a)
+{
+    uint32_t m = __vmaxu2(a.x & 0x7FFF7FFFu, a.y & 0x7FFF7FFFu);
+    m = __vmaxu2(m, __vmaxu2(a.z & 0x7FFF7FFFu, a.w & 0x7FFF7FFFu));
+    return m;
+}
+
+__device__ __forceinline__ float halves_max(uint32_t m)
+{
+    const uint32_t hi = m >> 16, lo = m & 0xFFFFu;
+    return __uint_as_float((hi > lo ? hi : lo) << 16);
+}
+
+__device__ __forceinline__ float global_scale_from_amax(uint32_t amax_bits)
+{
+    float s = __fdiv_rn(__uint_as_float(amax_bits), 2688.0f);
+    return (s >= 1.17549435e-38f) ? s : 1.0f;
+}
+
+// E4M3 code of t >= 0, round-to-nearest-even, saturating at 448 (hardware cvt).
+__device__ __forceinline__ uint32_t e4m3_code(float t)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(t));
+    return r & 0xFFu;
+}
+
+// Value of a non-negative finite E4M3 code (exact).
+__device__ __forceinline__ float e4m3_value(uint32_t c)
+{
+    const uint32_t e = c >> 3, m = c & 7u;
+    return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : (float)m * 0.001953125f;
+}
+
+// Eight E2M1 codes, element i in nibble i (hardware cvt: the second source
+// operand lands in the low nibble).
+__device__ __forceinline__ uint32_t e2m1x8(const float *y)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]),
+          "f"(y[7]));
+    return r;
+}
+
+// Clear the sign of every nibble whose magnitude is zero (no negative zero).
+__device__ __forceinline__ uint32_t drop_negative_zero(uint32_t w)
+{
+    const uint32_t mag = w & 0x77777777u;
+    const uint32_t nonzero = (mag + 0x77777777u) & 0x88888888u;
+    return mag | (w & nonzero);
+}
+
+__device__ __forceinline__ void unpack_bf16x8(uint4 a, float *x)
+{
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+// amax of the first chunk per (K/V, batch, head).  blockDim = (8H, ty),
+// grid = (gx, 2B).  amax must be zero on entry; float bits of non-negative
+// values order like unsigned integers, so atomicMax on the bits is exact.
+__global__ void k_first_chunk_amax(const uint4 *__restrict__ k, const uint4 *__restrict__ v,
+                                   uint32_t *__restrict__ amax, int B, int H, int Lq)
+{
+    __shared__ uint32_t s_max[64];
+    const int tid = threadIdx.y * blockDim.x + threadIdx.x;
+    if (tid < H) s_max[tid] = 0u;
+    __syncthreads();
+    const int t = blockIdx.y / B, b = blockIdx.y - t * B;
+    const uint4 *src = t ? v : k;
+    const int h = threadIdx.x >> 3, blk = threadIdx.x & 7;
+    uint32_t m = 0u;
+    for (int l = blockIdx.x * blockDim.y + threadIdx.y; l < Lq; l += gridDim.x * blockDim.y) {
+        const uint4 *p = src + (((size_t)b * Lq + l) * H + h) * 16 + blk * 2;
+        m = __vmaxu2(m, __vmaxu2(absmax_bits(ld_stream(p)), absmax_bits(ld_stream(p + 1))));
+    }
+    uint32_t f = __float_as_uint(halves_max(m));
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) {
+        const uint32_t g = __shfl_xor_sync(0xFFFFFFFFu, f, o);
+        f = g > f ? g : f;
+    }
+    if (blk == 0) atomicMax(&s_max[h], f);
+    __syncthreads();
+    if (tid < H && s_max[tid]) atomicMax(&amax[(t * B + b) * H + tid], s_max[tid]);
+}
+
+// blockDim = (8H, ty): threadIdx.x = h * 8 + block, threadIdx.y = token in the
+// CTA's token group.  grid = (ceil(Lq / ty), 2B): blockIdx.y = t * B + b with
+// t = 0 for K and 1 for V.
+__global__ void __launch_bounds__(512) k_nvfp4_append(const __grid_constant__ AppendLaunch a)
+{
+    const int t = blockIdx.y / a.B, b = blockIdx.y - t * a.B;
+    const int l = blockIdx.x * blockDim.y + threadIdx.y;
+    if (l >= a.Lq) return;
+    const int h = threadIdx.x >> 3, blk = threadIdx.x & 7;
+    const uint4 *src = reinterpret_cast<const uint4 *>(t ? a.v : a.k) +
+                       (((size_t)b * a.Lq + l) * a.H + h) * 16 + blk * 2;
+    const uint4 w0 = ld_stream(src), w1 = ld_stream(src + 1);
+
+    const int gi = (t * a.B + b) * a.H + h;
+    float sg;
+    if (a.first) {
+        sg = global_scale_from_amax(a.amax[gi]);
+        if (l == 0 && blk == 0) a.s_g[gi] = sg;
+    } else {
+        sg = a.s_g[gi];
+    }
+
+    const float amax16 = halves_max(__vmaxu2(absmax_bits(w0), absmax_bits(w1)));
+    const float ratio = __fdiv_rn(amax16, __fmul_rn(6.0f, sg));
+    const uint32_t sb_code = e4m3_code(ratio);
+    const float sb = e4m3_value(sb_code);
+    uint2 codes = make_uint2(0u, 0u);
+    if (sb != 0.0f) {
+        const float d = __fmul_rn(sb, sg);
+        float x[16], y[16];
+        unpack_bf16x8(w0, x);
+        unpack_bf16x8(w1, x + 8);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) y[i] = __fdiv_rn(x[i], d);
+        codes.x = drop_negative_zero(e2m1x8(y));
+        codes.y = drop_negative_zero(e2m1x8(y + 8));
+    }
+
+    const int frame = l / a.T, tok = l - frame * a.T;
+    const int slot = a.slot[b * a.C + frame];
+    const size_t row = (size_t)(b * a.H + h) * a.R + (size_t)slot * a.T + tok;
+    uint8_t *cdst = static_cast<uint8_t *>(t ? a.v_data : a.k_data) + row * 64 + blk * 8;
+    *reinterpret_cast<uint2 *>(cdst) = codes;
+    static_cast<uint8_t *>(t ? a.v_scales : a.k_scales)[row * 8 + blk] = (uint8_t)sb_code;
+}
+
+// bf16 twin: blockDim = (16H, ty), one 16-byte chunk per thread.
+__global__ void __launch_bounds__(1024) k_bf16_append(const __grid_constant__ AppendLaunch a)
+{
+    const int t = blockIdx.y / a.B, b = blockIdx.y - t * a.B;
+    const int l = blockIdx.x * blockDim.y + threadIdx.y;
+    if (l >= a.Lq) return;
+    const int h = threadIdx.x >> 4, c = threadIdx.x & 15;
+    const uint4 *src = reinterpret_cast<const uint4 *>(t ? a.v : a.k) +
+                       (((size_t)b * a.Lq + l) * a.H + h) * 16 + c;
+    const int frame = l / a.T, tok = l - frame * a.T;
+    const int slot = a.slot[b * a.C + frame];
+    const size_t row = (size_t)(b * a.H + h) * a.R + (size_t)slot * a.T + tok;
+    reinterpret_cast<uint4 *>(t ? a.v_data : a.k_data)[row * 16 + c] = ld_stream(src);
+}
+
+__global__ void k_encode_e2m1(const float *__restrict__ y, uint8_t *__restrict__ out, size_t n)
+{
+    const size_t i0 = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
+    if (i0 >= n) return;
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = (i0 + j < n) ? y[i0 + j] : 0.0f;
+    const uint32_t w = drop_negative_zero(e2m1x8(v));
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        if (i0 + j < n) out[i0 + j] = (w >> (4 * j)) & 15u;
+}
+
+__global__ void k_encode_block_scale(const float *__restrict__ t, uint8_t *__restrict__ out,
+                                     size_t n)
+{
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) out[i] = (uint8_t)e4m3_code(t[i]);
+}
+
+dim3 append_block(int H, int per_head)
+{
+    const int x = per_head * H;
+    const int y = x >= 256 ? 1 : 256 / x;
+    return dim3(x, y);
+}
+
+}  // namespace
+
+cudaError_t launch_nvfp4_append(const AppendLaunch &a, cudaStream_t s)
+{
+    const dim3 blk = append_block(a.H, 8);
+    const dim3 grid((a.Lq + blk.y - 1) / blk.y, 2 * a.B);
+    if (a.first) {
+        cudaError_t e = cudaMemsetAsync(a.amax, 0, sizeof(uint32_t) * 2 * a.B * a.H, s);
+        if (e != cudaSuccess) return e;
+        const dim3 g2(grid.x < 148 ? grid.x : 148, 2 * a.B);
+        k_first_chunk_amax<<<g2, blk, 0, s>>>(static_cast<const uint4 *>(a.k),
+                                              static_cast<const uint4 *>(a.v), a.amax, a.B, a.H,
+                                              a.Lq);
+    }
+    k_nvfp4_append<<<grid, blk, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bf16_append(const AppendLaunch &a, cudaStream_t s)
+{
+    const dim3 blk = append_block(a.H, 16);
+    const dim3 grid((a.Lq + blk.y - 1) / blk.y, 2 * a.B);
+    k_bf16_append<<<grid, blk, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_encode_e2m1(const float *y, uint8_t *codes, size_t n, cudaStream_t s)
+{
+    const size_t groups = (n + 7) / 8;
+    k_encode_e2m1<<<(unsigned)((groups + 255) / 256), 256, 0, s>>>(y, codes, n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_encode_block_scale(const float *t, uint8_t *codes, size_t n, cudaStream_t s)
+{
+    k_encode_block_scale<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(t, codes, n);
+    return cudaGetLastError();
+}
+
+}  // namespace nvkv

@@ -1,0 +1,428 @@
+// C-ABI host layer: descriptor checks, cache sizing, the sink + rolling-window
+// ring, and the launch wrappers.  No device allocation, no host sync.
+//
+// Ring rules (attention sink and multi-shot sink: "NVlabs/LongLive 2.0: NVFP4
+// parallel infrastructure for long video generation", section "NVFP4,
+// sequence parallel and the async decode path"; relative RoPE: "NVlabs
+// LongLive" (refft.com), Core Analysis block "How do KV-cache relative RoPE
+// and TriAttention work together"):
+//   * capacity S + W frames, the window holding the current chunk;
+//   * the first S frames appended are the sink and stay resident;
+//   * eviction removes the oldest resident frames that are not sink and not
+//     pinned; a chunk goes into the lowest free physical slots;
+//   * logical order is sink first, then by age; the RoPE frame index of a
+//     resident frame is its logical index;
+//   * multi-shot: a chunk of shot s sees the global sink, every frame of shot
+//     s and the last frame of each earlier shot; the first chunk of a shot
+//     s > 0 is pinned while that shot runs.
+#include <cmath>
+#include <cstring>
+
+#include "nvkv_internal.h"
+
+namespace {
+
+using nvkv::AppendLaunch;
+using nvkv::AttnLaunch;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+nvkv_status check_desc(const nvkv_desc *d)
+{
+    if (!d) return NVKV_ERR_INVALID_ARG;
+    if (d->magic != NVKV_MAGIC || d->version != NVKV_VERSION) return NVKV_ERR_STATE;
+    if (d->D != NVKV_HEAD_DIM) return NVKV_ERR_UNSUPPORTED;
+    if (d->B < 1 || d->H < 1 || d->grid_h < 1 || d->grid_w < 1 || d->C < 1 || d->S < 0 ||
+        d->W < 1)
+        return NVKV_ERR_INVALID_ARG;
+    if (d->B > NVKV_MAX_BATCH || d->H > 64 || d->C > NVKV_MAX_CHUNK || d->C > d->W ||
+        d->S + d->W > NVKV_MAX_FRAMES || d->grid_h > 65535 || d->grid_w > 65535)
+        return NVKV_ERR_UNSUPPORTED;
+    if (d->kv_dtype != NVKV_KV_NVFP4 && d->kv_dtype != NVKV_KV_BF16) return NVKV_ERR_INVALID_ARG;
+    if (d->rope_split[0] + d->rope_split[1] + d->rope_split[2] != NVKV_HEAD_DIM ||
+        (d->rope_split[0] | d->rope_split[1] | d->rope_split[2]) & 1 || d->rope_split[0] < 0 ||
+        d->rope_split[1] < 0 || d->rope_split[2] < 0 || !(d->rope_base > 0.0f))
+        return NVKV_ERR_INVALID_ARG;
+    const int64_t T = (int64_t)d->grid_h * d->grid_w;
+    const int64_t R = T * (d->S + d->W);
+    // 32-bit index arithmetic in the kernels
+    if (R * d->B * d->H * 128 >= (int64_t(1) << 31) / 2 ||
+        T * d->C * d->B * d->H * 128 >= (int64_t(1) << 31) / 2)
+        return NVKV_ERR_UNSUPPORTED;
+    return NVKV_OK;
+}
+
+nvkv_status check_ring(const nvkv_desc *d, const nvkv_ring *r)
+{
+    if (!r) return NVKV_ERR_INVALID_ARG;
+    if (r->magic != NVKV_MAGIC || r->version != NVKV_VERSION) return NVKV_ERR_STATE;
+    if (r->B != d->B || r->capacity != d->S + d->W || r->C != d->C || r->S != d->S)
+        return NVKV_ERR_STATE;
+    for (int b = 0; b < d->B; ++b)
+        if (r->s[b].n_resident < 0 || r->s[b].n_resident > r->capacity) return NVKV_ERR_STATE;
+    return NVKV_OK;
+}
+
+int64_t rows_per_head(const nvkv_desc *d) { return (int64_t)d->grid_h * d->grid_w * (d->S + d->W); }
+
+bool is_visible(const nvkv_ring_stream &s, int i)
+{
+    return (s.flags[i] & (NVKV_FRAME_SINK | NVKV_FRAME_SHOT_LAST)) || s.frame_shot[i] == s.shot;
+}
+
+// Assigns C free physical slots to every stream; fills a.slot.  Does not
+// modify the ring.  Returns false if some stream has no room.
+bool plan_slots(const nvkv_desc *d, const nvkv_ring *r, int32_t *slot_out)
+{
+    const int cap = d->S + d->W;
+    for (int b = 0; b < d->B; ++b) {
+        const nvkv_ring_stream &s = r->s[b];
+        if (s.n_resident + d->C > cap) return false;
+        bool used[NVKV_MAX_FRAMES] = {};
+        for (int i = 0; i < s.n_resident; ++i) used[s.slot[i]] = true;
+        int c = 0;
+        for (int p = 0; p < cap && c < d->C; ++p)
+            if (!used[p]) slot_out[b * d->C + c++] = p;
+        if (c < d->C) return false;
+    }
+    return true;
+}
+
+void commit_append(const nvkv_desc *d, nvkv_ring *r, const int32_t *slot)
+{
+    for (int b = 0; b < d->B; ++b) {
+        nvkv_ring_stream &s = r->s[b];
+        for (int c = 0; c < d->C; ++c) {
+            const int i = s.n_resident++;
+            const int fno = s.n_appended++;
+            s.slot[i] = slot[b * d->C + c];
+            s.frame[i] = fno;
+            s.frame_shot[i] = s.shot;
+            s.flags[i] = (fno < d->S ? NVKV_FRAME_SINK : 0u) | (s.pin_next ? NVKV_FRAME_PINNED : 0u);
+        }
+        s.pin_next = 0;
+    }
+    r->scales_fixed = 1;
+    r->steps += 1;
+}
+
+nvkv_status append_common(const nvkv_desc *desc, const nvkv_cache *cache, nvkv_ring *ring,
+                          const void *k, const void *v, cudaStream_t stream, int dtype)
+{
+    nvkv_status st = check_desc(desc);
+    if (st != NVKV_OK) return st;
+    if (desc->kv_dtype != dtype) return NVKV_ERR_STATE;
+    if ((st = check_ring(desc, ring)) != NVKV_OK) return st;
+    if (!cache || !k || !v || !cache->k_data || !cache->v_data) return NVKV_ERR_INVALID_ARG;
+    if (dtype == NVKV_KV_NVFP4 &&
+        (!cache->k_scales || !cache->v_scales || !cache->amax || !cache->s_g))
+        return NVKV_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(cache->k_data) || !aligned16(cache->v_data) ||
+        (dtype == NVKV_KV_NVFP4 && (!aligned16(cache->k_scales) || !aligned16(cache->v_scales))))
+        return NVKV_ERR_ALIGNMENT;
+
+    AppendLaunch a{};
+    if (!plan_slots(desc, ring, a.slot)) return NVKV_ERR_CAPACITY;
+    a.k = k;
+    a.v = v;
+    a.k_data = cache->k_data;
+    a.v_data = cache->v_data;
+    a.k_scales = cache->k_scales;
+    a.v_scales = cache->v_scales;
+    a.amax = cache->amax;
+    a.s_g = cache->s_g;
+    a.B = desc->B;
+    a.H = desc->H;
+    a.T = desc->grid_h * desc->grid_w;
+    a.Lq = desc->C * a.T;
+    a.R = (int)rows_per_head(desc);
+    a.C = desc->C;
+    a.first = ring->scales_fixed ? 0 : 1;
+    cudaError_t e = (dtype == NVKV_KV_NVFP4) ? nvkv::launch_nvfp4_append(a, stream)
+                                             : nvkv::launch_bf16_append(a, stream);
+    if (e != cudaSuccess) return NVKV_ERR_CUDA;
+    commit_append(desc, ring, a.slot);
+    return NVKV_OK;
+}
+
+nvkv_status attention_common(const nvkv_desc *desc, const nvkv_cache *cache,
+                             const nvkv_ring *ring, const void *q, void *out, float *lse,
+                             void *ws, size_t ws_bytes, cudaStream_t stream, int dtype)
+{
+    (void)ws;
+    (void)ws_bytes;
+    nvkv_status st = check_desc(desc);
+    if (st != NVKV_OK) return st;
+    if (desc->kv_dtype != dtype) return NVKV_ERR_STATE;
+    if ((st = check_ring(desc, ring)) != NVKV_OK) return st;
+    if (ring->steps < 1) return NVKV_ERR_STATE;
+    if (!cache || !q || !out || !cache->k_data || !cache->v_data || !cache->status)
+        return NVKV_ERR_INVALID_ARG;
+    if (dtype == NVKV_KV_NVFP4 && (!cache->k_scales || !cache->v_scales || !cache->s_g))
+        return NVKV_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(out) || !aligned16(cache->k_data) ||
+        !aligned16(cache->v_data) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
+        (dtype == NVKV_KV_NVFP4 && (!aligned16(cache->k_scales) || !aligned16(cache->v_scales))))
+        return NVKV_ERR_ALIGNMENT;
+
+    AttnLaunch a{};
+    a.q = q;
+    a.out = out;
+    a.lse = lse;
+    a.k_data = cache->k_data;
+    a.v_data = cache->v_data;
+    a.k_scales = cache->k_scales;
+    a.v_scales = cache->v_scales;
+    a.s_g = cache->s_g;
+    a.status = cache->status;
+    a.B = desc->B;
+    a.H = desc->H;
+    a.T = desc->grid_h * desc->grid_w;
+    a.Lq = desc->C * a.T;
+    a.R = (int)rows_per_head(desc);
+    a.grid_w = desc->grid_w;
+    a.kv_dtype = dtype;
+    a.grid_h = desc->grid_h;
+    // the attention kernels are built for the 44/42/42 split and small grids
+    if (desc->rope_split[0] != 44 || desc->rope_split[1] != 42 || desc->rope_split[2] != 42 ||
+        desc->grid_h > 256 || desc->grid_w > 256)
+        return NVKV_ERR_UNSUPPORTED;
+    {
+        int p = 0;
+        for (int ax = 0; ax < 3; ++ax) {
+            const int d = desc->rope_split[ax];
+            for (int i = 0; i < d / 2; ++i)
+                a.theta[p++] = (float)std::pow((double)desc->rope_base, -2.0 * i / (double)d);
+        }
+    }
+    a.n_fpos = 0;
+    for (int b = 0; b < desc->B; ++b) {
+        const nvkv_ring_stream &s = ring->s[b];
+        if (s.n_resident < desc->C) return NVKV_ERR_STATE;
+        int n = 0;
+        for (int i = 0; i < s.n_resident; ++i)
+            if (is_visible(s, i)) {
+                a.vis[b][n].slot = (uint16_t)s.slot[i];
+                a.vis[b][n].rope_pos = (uint16_t)i;
+                ++n;
+            }
+        a.n_vis[b] = n;
+        a.q_pos0[b] = s.n_resident - desc->C;
+        if (s.n_resident > a.n_fpos) a.n_fpos = s.n_resident;
+    }
+    if (nvkv::launch_chunk_attention(a, stream) != cudaSuccess) return NVKV_ERR_CUDA;
+    return NVKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+nvkv_status nvkv_desc_init(nvkv_desc *desc, int B, int H, int grid_h, int grid_w, int C, int S,
+                           int W, int kv_dtype)
+{
+    if (!desc) return NVKV_ERR_INVALID_ARG;
+    std::memset(desc, 0, sizeof(*desc));
+    desc->magic = NVKV_MAGIC;
+    desc->version = NVKV_VERSION;
+    desc->B = B;
+    desc->H = H;
+    desc->D = NVKV_HEAD_DIM;
+    desc->grid_h = grid_h;
+    desc->grid_w = grid_w;
+    desc->C = C;
+    desc->S = S;
+    desc->W = W;
+    desc->kv_dtype = kv_dtype;
+    desc->rope_base = 10000.0f;
+    desc->rope_split[0] = 44;
+    desc->rope_split[1] = 42;
+    desc->rope_split[2] = 42;
+    return check_desc(desc);
+}
+
+size_t nvkv_plane_bytes(const nvkv_desc *d, int plane)
+{
+    if (check_desc(d) != NVKV_OK) return 0;
+    const size_t rows = (size_t)rows_per_head(d) * d->B * d->H;
+    const bool fp4 = d->kv_dtype == NVKV_KV_NVFP4;
+    switch (plane) {
+    case NVKV_PLANE_K_DATA:
+    case NVKV_PLANE_V_DATA: return rows * (fp4 ? 64 : 256);
+    // +16 bytes: scale runs are copied in 16-byte granules that may reach one
+    // row past the last one
+    case NVKV_PLANE_K_SCALES:
+    case NVKV_PLANE_V_SCALES: return fp4 ? rows * 8 + 16 : 0;
+    case NVKV_PLANE_AMAX: return fp4 ? sizeof(uint32_t) * 2 * d->B * d->H : 0;
+    case NVKV_PLANE_SCALE_G: return fp4 ? sizeof(float) * 2 * d->B * d->H : 0;
+    case NVKV_PLANE_STATUS: return sizeof(int32_t);
+    default: return 0;
+    }
+}
+
+nvkv_status nvkv_ring_init(const nvkv_desc *desc, nvkv_ring *ring)
+{
+    nvkv_status st = check_desc(desc);
+    if (st != NVKV_OK) return st;
+    if (!ring) return NVKV_ERR_INVALID_ARG;
+    std::memset(ring, 0, sizeof(*ring));
+    ring->magic = NVKV_MAGIC;
+    ring->version = NVKV_VERSION;
+    ring->B = desc->B;
+    ring->capacity = desc->S + desc->W;
+    ring->C = desc->C;
+    ring->S = desc->S;
+    return NVKV_OK;
+}
+
+nvkv_status kv_ring_evict(const nvkv_desc *desc, nvkv_ring *ring, int n_frames)
+{
+    nvkv_status st = check_desc(desc);
+    if (st != NVKV_OK) return st;
+    if ((st = check_ring(desc, ring)) != NVKV_OK) return st;
+    if (n_frames < 0) return NVKV_ERR_INVALID_ARG;
+    for (int b = 0; b < desc->B; ++b) {
+        const nvkv_ring_stream &s = ring->s[b];
+        int n = 0;
+        for (int i = 0; i < s.n_resident; ++i)
+            if (!(s.flags[i] & (NVKV_FRAME_SINK | NVKV_FRAME_PINNED))) ++n;
+        if (n < n_frames) return NVKV_ERR_CAPACITY;
+    }
+    for (int b = 0; b < desc->B; ++b) {
+        nvkv_ring_stream &s = ring->s[b];
+        int dropped = 0, w = 0;
+        for (int i = 0; i < s.n_resident; ++i) {
+            const bool evictable = !(s.flags[i] & (NVKV_FRAME_SINK | NVKV_FRAME_PINNED));
+            if (evictable && dropped < n_frames) {
+                ++dropped;
+                continue;
+            }
+            s.slot[w] = s.slot[i];
+            s.frame[w] = s.frame[i];
+            s.frame_shot[w] = s.frame_shot[i];
+            s.flags[w] = s.flags[i];
+            ++w;
+        }
+        s.n_resident = w;
+    }
+    return NVKV_OK;
+}
+
+nvkv_status kv_ring_begin_shot(const nvkv_desc *desc, nvkv_ring *ring, int b, int shot_id)
+{
+    nvkv_status st = check_desc(desc);
+    if (st != NVKV_OK) return st;
+    if ((st = check_ring(desc, ring)) != NVKV_OK) return st;
+    if (b < 0 || b >= desc->B) return NVKV_ERR_INVALID_ARG;
+    nvkv_ring_stream &s = ring->s[b];
+    if (shot_id < s.shot) return NVKV_ERR_INVALID_ARG;
+    if (shot_id == s.shot) return NVKV_OK;
+    if (s.n_resident > 0) s.flags[s.n_resident - 1] |= NVKV_FRAME_SHOT_LAST;
+    for (int i = 0; i < s.n_resident; ++i) s.flags[i] &= ~NVKV_FRAME_PINNED;
+    s.shot = shot_id;
+    s.pin_next = shot_id > 0 ? 1 : 0;
+    return NVKV_OK;
+}
+
+int nvkv_ring_visible(const nvkv_desc *desc, const nvkv_ring *ring, int b, int32_t *slots,
+                      int32_t *rope_pos, int32_t *frames, int32_t *query_pos0)
+{
+    if (check_desc(desc) != NVKV_OK || check_ring(desc, ring) != NVKV_OK || b < 0 || b >= desc->B)
+        return -1;
+    const nvkv_ring_stream &s = ring->s[b];
+    int n = 0;
+    for (int i = 0; i < s.n_resident; ++i)
+        if (is_visible(s, i)) {
+            if (slots) slots[n] = s.slot[i];
+            if (rope_pos) rope_pos[n] = i;
+            if (frames) frames[n] = s.frame[i];
+            ++n;
+        }
+    if (query_pos0) *query_pos0 = s.n_resident - desc->C;
+    return n;
+}
+
+nvkv_status nvkv_ring_push_chunk(const nvkv_desc *desc, nvkv_ring *ring, int32_t *slots_out)
+{
+    nvkv_status st = check_desc(desc);
+    if (st != NVKV_OK) return st;
+    if ((st = check_ring(desc, ring)) != NVKV_OK) return st;
+    int32_t slot[NVKV_MAX_BATCH * NVKV_MAX_CHUNK];
+    if (!plan_slots(desc, ring, slot)) return NVKV_ERR_CAPACITY;
+    commit_append(desc, ring, slot);
+    if (slots_out) std::memcpy(slots_out, slot, sizeof(int32_t) * desc->B * desc->C);
+    return NVKV_OK;
+}
+
+nvkv_status nvfp4_kv_append(const nvkv_desc *desc, const nvkv_cache *cache, nvkv_ring *ring,
+                            const void *k, const void *v, nvkv_stream stream)
+{
+    return append_common(desc, cache, ring, k, v, (cudaStream_t)stream, NVKV_KV_NVFP4);
+}
+
+nvkv_status bf16_kv_append(const nvkv_desc *desc, const nvkv_cache *cache, nvkv_ring *ring,
+                           const void *k, const void *v, nvkv_stream stream)
+{
+    return append_common(desc, cache, ring, k, v, (cudaStream_t)stream, NVKV_KV_BF16);
+}
+
+size_t nvkv_attention_workspace_bytes(const nvkv_desc *desc)
+{
+    (void)desc;
+    return 0;
+}
+
+nvkv_status chunk_attention_nvfp4kv(const nvkv_desc *desc, const nvkv_cache *cache,
+                                    const nvkv_ring *ring, const void *q, void *out, float *lse,
+                                    void *workspace, size_t workspace_bytes, nvkv_stream stream)
+{
+    return attention_common(desc, cache, ring, q, out, lse, workspace, workspace_bytes,
+                            (cudaStream_t)stream, NVKV_KV_NVFP4);
+}
+
+nvkv_status chunk_attention_bf16kv(const nvkv_desc *desc, const nvkv_cache *cache,
+                                   const nvkv_ring *ring, const void *q, void *out, float *lse,
+                                   void *workspace, size_t workspace_bytes, nvkv_stream stream)
+{
+    return attention_common(desc, cache, ring, q, out, lse, workspace, workspace_bytes,
+                            (cudaStream_t)stream, NVKV_KV_BF16);
+}
+
+nvkv_status nvkv_encode_e2m1(const float *y, uint8_t *codes, size_t n, nvkv_stream stream)
+{
+    if (n == 0) return NVKV_OK;
+    if (!y || !codes) return NVKV_ERR_INVALID_ARG;
+    if (n > (size_t(1) << 31)) return NVKV_ERR_UNSUPPORTED;
+    return nvkv::launch_encode_e2m1(y, codes, n, (cudaStream_t)stream) == cudaSuccess
+               ? NVKV_OK
+               : NVKV_ERR_CUDA;
+}
+
+nvkv_status nvkv_encode_block_scale(const float *t, uint8_t *codes, size_t n, nvkv_stream stream)
+{
+    if (n == 0) return NVKV_OK;
+    if (!t || !codes) return NVKV_ERR_INVALID_ARG;
+    if (n > (size_t(1) << 31)) return NVKV_ERR_UNSUPPORTED;
+    return nvkv::launch_encode_block_scale(t, codes, n, (cudaStream_t)stream) == cudaSuccess
+               ? NVKV_OK
+               : NVKV_ERR_CUDA;
+}
+
+const char *nvkv_status_string(nvkv_status s)
+{
+    switch (s) {
+    case NVKV_OK: return "ok";
+    case NVKV_ERR_INVALID_ARG: return "invalid argument";
+    case NVKV_ERR_UNSUPPORTED: return "unsupported shape or device";
+    case NVKV_ERR_ALIGNMENT: return "device pointer not 16-byte aligned";
+    case NVKV_ERR_CAPACITY: return "no room in the ring (evict first) or too few evictable frames";
+    case NVKV_ERR_STATE: return "descriptor/ring/cache state mismatch";
+    case NVKV_ERR_CUDA: return "CUDA launch failed";
+    case NVKV_ERR_TIMEOUT: return "device pipeline wait exceeded its bound";
+    }
+    return "unknown status";
+}
+
+uint32_t nvkv_version(void) { return NVKV_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,56 @@
+// Internal launch interface between the C-ABI host layer (nvkv_host.cpp) and
+// the CUDA kernels (append.cu, attention.cu).  Not part of the public ABI.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/nvkv.h"
+
+namespace nvkv {
+
+// Quantize-append / bf16 append of one chunk into physical frame slots.
+struct AppendLaunch {
+    const void *k, *v;               // bf16 [B][Lq][H][128]
+    void *k_data, *v_data;           // NVFP4 codes [B][H][R][64] or bf16 [B][H][R][128]
+    void *k_scales, *v_scales;       // E4M3 [B][H][R][8] (NVFP4 only)
+    uint32_t *amax;                  // [2][B][H]
+    float *s_g;                      // [2][B][H]
+    int B, H, T, Lq, R, C;
+    int first;                       // 1: measure amax and fix s_g
+    int32_t slot[NVKV_MAX_BATCH * NVKV_MAX_CHUNK];  // [b * C + c] -> physical slot
+};
+
+cudaError_t launch_nvfp4_append(const AppendLaunch &a, cudaStream_t s);
+cudaError_t launch_bf16_append(const AppendLaunch &a, cudaStream_t s);
+cudaError_t launch_encode_e2m1(const float *y, uint8_t *codes, size_t n, cudaStream_t s);
+cudaError_t launch_encode_block_scale(const float *t, uint8_t *codes, size_t n, cudaStream_t s);
+
+// One visible frame of a stream: physical slot and RoPE frame index.
+struct VisFrame {
+    uint16_t slot;
+    uint16_t rope_pos;
+};
+
+// Chunk attention over the visible frames of every stream.
+struct AttnLaunch {
+    const void *q;                   // bf16 [B][Lq][H][128]
+    void *out;                       // bf16 [B][Lq][H][128]
+    float *lse;                      // f32 [B][H][Lq] or null
+    const void *k_data, *v_data;
+    const void *k_scales, *v_scales;
+    const float *s_g;                // [2][B][H] (NVFP4 only)
+    int32_t *status;
+    int B, H, T, Lq, R, grid_w;
+    int kv_dtype;
+    int n_vis[NVKV_MAX_BATCH];       // visible frames per stream
+    int q_pos0[NVKV_MAX_BATCH];      // RoPE frame index of the chunk's first frame
+    VisFrame vis[NVKV_MAX_BATCH][NVKV_MAX_FRAMES];
+    int grid_h;
+    int n_fpos;                      // frame positions used: 0 .. n_fpos-1
+    float theta[64];                 // RoPE angle per unit position of each channel pair
+};
+
+cudaError_t launch_chunk_attention(const AttnLaunch &a, cudaStream_t s);
+
+}  // namespace nvkv

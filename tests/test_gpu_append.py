@@ -1,0 +1,117 @@
+"""Quantize-append parity: every code and scale byte the CUDA path writes
+equals the oracle's, at every step, in the physical slot the ring assigned;
+nothing outside those slots is touched."""
+import numpy as np
+import pytest
+import torch
+
+import kvsynth
+import oracle
+from oracle.stream import OracleStream
+from tests._harness import LibStream, to_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_new_frames(lib: LibStream, ora: OracleStream, new):
+    wl = lib.wl
+    for b, fids in new.items():
+        for fid in fids:
+            rows = lib.frame_rows(b, fid)
+            e = ora.frame(b, fid)
+            for w in ("k", "v"):
+                got_c = lib.cache.codes(w)[b, :, rows].cpu().numpy()
+                got_s = lib.cache.scales(w)[b, :, rows].cpu().numpy()
+                assert np.array_equal(got_c, e[w + "_codes"]), (b, fid, w)
+                assert np.array_equal(got_s, e[w + "_scales"]), (b, fid, w)
+
+
+@pytest.mark.parametrize("name", ["tiny", "stream1p3b", "stream5b"])
+def test_append_bit_exact(name):
+    import nvfp4_kv_cache_append_b200 as nv
+    wl = kvsynth.WORKLOADS[name]
+    lib = LibStream(wl, nv.NVKV_KV_NVFP4)
+    ora = OracleStream(wl, seed=0, keep_inputs=False)
+    for step in range(1, wl.steps + 1):
+        x = kvsynth.chunk_qkv(wl, step, 0)
+        new = ora.step(k=x["k"], v=x["v"], q=x["q"])
+        g = to_gpu(x)
+        lib.step(g["q"], g["k"], g["v"])
+        torch.cuda.synchronize()
+        if step == 1:
+            assert np.array_equal(lib.cache.global_scales().cpu().numpy(), ora.s_g)
+        _check_new_frames(lib, ora, new)
+    assert lib.cache.device_status() == 0
+    # after the ring wrapped, every resident frame still matches
+    for b in range(wl.B):
+        for fid in ora.rings[b].resident():
+            _check_new_frames(lib, ora, {b: [fid]})
+
+
+def test_append_multishot_bit_exact():
+    import nvfp4_kv_cache_append_b200 as nv
+    wl = kvsynth.WORKLOADS["multishot"]
+    sched = kvsynth.shot_schedule(wl, 0)
+    lib = LibStream(wl, nv.NVKV_KV_NVFP4, sched=sched)
+    ora = OracleStream(wl, seed=0, shot_sched=sched, keep_inputs=False)
+    for step in range(1, wl.steps + 1):
+        x = kvsynth.chunk_qkv(wl, step, 0)
+        new = ora.step(k=x["k"], v=x["v"], q=x["q"])
+        g = to_gpu(x)
+        lib.step(g["q"], g["k"], g["v"], with_lse=False)
+        torch.cuda.synchronize()
+        if step in (1, 2, 9, 16, 17, 24):
+            _check_new_frames(lib, ora, new)
+        for b in range(wl.B):
+            assert lib.cache.visible(b)[2] == [f for f, _ in ora.rings[b].visible()]
+
+
+def test_append_leaves_other_bytes_alone():
+    import nvfp4_kv_cache_append_b200 as nv
+    wl = kvsynth.WORKLOADS["tiny"]
+    lib = LibStream(wl, nv.NVKV_KV_NVFP4)
+    for t in (lib.cache.k_data, lib.cache.v_data, lib.cache.k_scales, lib.cache.v_scales):
+        t.fill_(0xA5)
+    x = to_gpu(kvsynth.chunk_qkv(wl, 1, 0))
+    lib.step(x["q"], x["k"], x["v"])
+    torch.cuda.synchronize()
+    rows = lib.frame_rows(0, 0)
+    for w in ("k", "v"):
+        c = lib.cache.codes(w)[0].clone()
+        s = lib.cache.scales(w)[0].clone()
+        c[:, rows] = 0xA5
+        s[:, rows] = 0xA5
+        assert bool((c == 0xA5).all()) and bool((s == 0xA5).all())
+    pad = lib.cache.k_scales[-16:]
+    assert bool((pad == 0xA5).all())
+
+
+def test_zero_first_chunk_gives_unit_scale_and_zero_codes():
+    import nvfp4_kv_cache_append_b200 as nv
+    wl = kvsynth.WORKLOADS["tiny"]
+    lib = LibStream(wl, nv.NVKV_KV_NVFP4)
+    z = torch.zeros(wl.B, wl.Lq, wl.H, 128, dtype=torch.bfloat16, device="cuda")
+    lib.step(z, z, z)
+    torch.cuda.synchronize()
+    assert bool((lib.cache.global_scales() == 1.0).all())
+    rows = lib.frame_rows(0, 0)
+    assert int(lib.cache.codes("k")[0, :, rows].sum()) == 0
+    assert int(lib.cache.scales("v")[0, :, rows].sum()) == 0
+
+
+def test_bf16_twin_append_copies_exactly():
+    import nvfp4_kv_cache_append_b200 as nv
+    wl = kvsynth.WORKLOADS["stream5b"]
+    lib = LibStream(wl, nv.NVKV_KV_BF16)
+    for step in range(1, wl.steps + 1):
+        x = kvsynth.chunk_qkv(wl, step, 0)
+        g = to_gpu(x)
+        lib.step(g["q"], g["k"], g["v"], with_lse=False)
+        torch.cuda.synchronize()
+        for c in range(wl.C):
+            fid = (step - 1) * wl.C + c
+            rows = lib.frame_rows(0, fid)
+            for w in ("k", "v"):
+                want = x[w][0, c * wl.T:(c + 1) * wl.T].transpose(0, 1)
+                got = lib.cache.codes(w)[0, :, rows].cpu()
+                assert torch.equal(got.view(torch.int16), want.contiguous().view(torch.int16))
