@@ -232,7 +232,9 @@ NVKV_API nvkv_status chunk_attention_nvfp4kv(const nvkv_desc *desc, const nvkv_c
                                     const nvkv_ring *ring, const void *q, void *out, float *lse,
                                     void *workspace, size_t workspace_bytes, nvkv_stream stream);
 
-/* The bf16-KV twin of chunk_attention_nvfp4kv. */
+/* The bf16-KV twin of chunk_attention_nvfp4kv.  Both attention calls feed the
+ * tensor cores f16 operands with f32 accumulation; the twin therefore needs
+ * cached K/V and rotated Q/K inside the f16 range (|x| < 65504). */
 NVKV_API nvkv_status chunk_attention_bf16kv(const nvkv_desc *desc, const nvkv_cache *cache,
                                    const nvkv_ring *ring, const void *q, void *out, float *lse,
                                    void *workspace, size_t workspace_bytes, nvkv_stream stream);

@@ -24,8 +24,8 @@
 //              S_j = Q K_j^T and O += P_j V_j with tcgen05.mma kind::f16,
 //              M = N = 128, accumulators in TMEM (S double buffered, O single).
 // The global scales are folded out of the dequantization: s_g(K) goes into the
-// softmax scale, s_g(V) into the epilogue.  The NVFP4 path computes in f16
-// operands (dequantized K/V are exact there), the bf16 twin in bf16.
+// softmax scale, s_g(V) into the epilogue.  Both caches compute with f16
+// operands (dequantized NVFP4 values are exact there).
 // Every mbarrier wait is bounded; on expiry the CTA records NVKV_ERR_TIMEOUT
 // in the status word, unwinds, waits for its own MMAs and frees TMEM.
 #include <cuda_bf16.h>
@@ -132,18 +132,15 @@ __device__ __forceinline__ uint32_t as_u(__half2 h) { return *reinterpret_cast<u
 // RoPE table entry.  NVFP4 path: (c, c) and (-s, s) as f16x2; bf16 twin: (c, s) f32.
 struct RopeH { uint32_t cc, ns; };
 
-template <bool FP4>
-struct Cfg;
-template <>
-struct Cfg<true> { static constexpr uint32_t fmt = 0; };   // f16 operands
-template <>
-struct Cfg<false> { static constexpr uint32_t fmt = 1; };  // bf16 operands
+// Both caches feed the tensor cores f16 operands (kind::f16, f32 accumulate).
+// NVFP4: code * s_b is exact in f16.  bf16 twin: cached values convert to f16
+// exactly inside f16's normal range (|x| in [2^-14, 65504]); rotated keys,
+// queries and probabilities keep 3 more mantissa bits than bf16 would.
+constexpr uint32_t kOperandF16 = 0;
 
-__device__ __forceinline__ uint32_t pack2(float lo, float hi, bool f16)
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi)
 {
-    if (f16) return as_u(__floats2half2_rn(lo, hi));
-    __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&b);
+    return as_u(__floats2half2_rn(lo, hi));
 }
 
 struct Ctx {
@@ -255,7 +252,7 @@ __device__ void load_q(Ctx &c, int r)
             const float x = __uint_as_float(u[k] << 16), y = __uint_as_float(u[k] & 0xFFFF0000u);
             float cs, sn;
             rope_cs_f32(c, FP4, rope_entry(c, p, fpos, hp, wp), cs, sn);
-            o[k] = pack2(x * cs - y * sn, x * sn + y * cs, FP4);
+            o[k] = pack_f16(x * cs - y * sn, x * sn + y * cs);
         }
         sts16(qs + swz(r, ch), o[0], o[1], o[2], o[3]);
     }
@@ -360,10 +357,15 @@ __device__ void convert_bf16_row(const Ctx &c, int r, const KeyRow &k, uint32_t 
             const float x = __uint_as_float(u[q] << 16), y = __uint_as_float(u[q] & 0xFFFF0000u);
             float cs, sn;
             rope_cs_f32(c, false, rope_entry(c, p, k.fpos, k.hp, k.wp), cs, sn);
-            o[q] = pack2(x * cs - y * sn, x * sn + y * cs, false);
+            o[q] = pack_f16(x * cs - y * sn, x * sn + y * cs);
         }
+        const uint32_t vu[4] = {vw.x, vw.y, vw.z, vw.w};
+        uint32_t vo[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            vo[q] = pack_f16(__uint_as_float(vu[q] << 16), __uint_as_float(vu[q] & 0xFFFF0000u));
         sts16(kdst + swz(r, ch), o[0], o[1], o[2], o[3]);
-        sts16(vdst + swz(r, ch), vw.x, vw.y, vw.z, vw.w);
+        sts16(vdst + swz(r, ch), vo[0], vo[1], vo[2], vo[3]);
     }
 }
 
@@ -412,8 +414,8 @@ __device__ void mma_role(Ctx &c)
     const uint32_t tmem = c.ctl->tmem_base;
     const uint32_t tS[2] = {tmem, tmem + 128};
     const uint32_t tO = tmem + 256;
-    constexpr uint32_t idS = ptx::idesc_f16(Cfg<FP4>::fmt, BM, BN, 0);
-    constexpr uint32_t idO = ptx::idesc_f16(Cfg<FP4>::fmt, BM, 128, 1);
+    constexpr uint32_t idS = ptx::idesc_f16(kOperandF16, BM, BN, 0);
+    constexpr uint32_t idO = ptx::idesc_f16(kOperandF16, BM, 128, 1);
     const uint32_t qs = ptx::smem_u32(c.smem + OFF_Q);
     const uint32_t ks = ptx::smem_u32(c.smem + OFF_K);
     const uint32_t vs = ptx::smem_u32(c.smem + OFF_V);
@@ -514,7 +516,7 @@ __device__ void softmax_role(Ctx &c)
             const float p0 = (2 * i < nv) ? ex2(s[2 * i] * scale - m) : 0.0f;
             const float p1 = (2 * i + 1 < nv) ? ex2(s[2 * i + 1] * scale - m) : 0.0f;
             l += p0 + p1;
-            pk[i] = pack2(p0, p1, FP4);
+            pk[i] = pack_f16(p0, p1);
         }
         if (j > 0 && !(ok = wait_warp(c, B_ODONE, (j - 1) & 1))) break;
 #pragma unroll

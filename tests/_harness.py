@@ -6,6 +6,9 @@ fp64 oracle run on the same dequantized K/V and bf16 Q.
 """
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -26,6 +29,11 @@ def parity(got: np.ndarray, ref: np.ndarray):
 
 def assert_parity(got, ref, what=""):
     max_abs, rel = parity(got, ref)
+    log = os.environ.get("NVKV_PARITY_LOG")
+    if log:
+        with open(log, "a") as f:
+            f.write(json.dumps({"case": os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0],
+                                "what": what, "max_abs": max_abs, "rel_l2": rel}) + "\n")
     assert np.isfinite(got).all(), what
     assert max_abs <= TOL_MAX_ABS and rel <= TOL_REL_L2, f"{what}: max_abs {max_abs:.3e} rel_l2 {rel:.3e}"
     return max_abs, rel
