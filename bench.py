@@ -39,6 +39,26 @@ def _peaks():
             "source": "fallback"}
 
 
+def _ncu_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu capture, or None when the
+    kernel's sources changed since the counters were taken."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f).get(kernel)
+    if not d:
+        return None
+    h = hashlib.sha256()
+    for src in d["sources"]:
+        with open(os.path.join(ROOT, src), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest()[:16] != d["source_sha256_16"]:
+        return None
+    return d["dram_bytes_read"] + d["dram_bytes_write"]
+
+
 def workload_numbers(wl):
     """Algorithmic work per step (see the per-kernel accounting in the docs)."""
     T, Lq = wl.T, wl.Lq
@@ -264,7 +284,8 @@ def run_ours(args):
         "append_gbs": append_gbs,
         "append_ms": app_avg,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak,
-                     "unit": "TFLOP/s", "frac": attn_tflops / peak, "traffic": None,
+                     "unit": "TFLOP/s", "frac": attn_tflops / peak,
+                     "traffic": _ncu_traffic("k_chunk_attn<1>") if fp4 else None,
                      "kernel": "k_chunk_attn", "peak_source": peaks["source"] + " bf16 (f16 same nominal rate)"},
         "append_roofline": {"bound": "hbm", "achieved": append_gbs, "peak": peaks["hbm_gbs"],
                             "unit": "GB/s", "frac": append_gbs / peaks["hbm_gbs"]},
