@@ -213,6 +213,25 @@ NVKV_API nvkv_status nvkv_ring_push_chunk(const nvkv_desc *desc, nvkv_ring *ring
 NVKV_API nvkv_status nvfp4_kv_append(const nvkv_desc *desc, const nvkv_cache *cache, nvkv_ring *ring,
                             const void *k, const void *v, nvkv_stream stream);
 
+/* nvfp4_kv_append for callers that cannot allocate device memory (no
+ * counterpart in the paper; an interface addition of this library).  The
+ * regular call needs the small caller-allocated scratch plane cache->amax,
+ * where the first append reduces each head's absolute maximum.  An
+ * inference-engine plugin whose enqueue step may not allocate, or a process
+ * whose device memory is all owned by another allocator, cannot provide it.
+ * This call keeps that scratch in a fixed array inside the library's device
+ * image instead (2 KiB; every GPU that loads the library holds it until the
+ * process exits) and allocates nothing.  Same inputs, outputs, slot logic and
+ * results as nvfp4_kv_append; cache->amax is ignored and may be NULL.
+ *  - B * H must be <= 256, else NVKV_ERR_UNSUPPORTED.
+ *  - The first call on a device sets up the array's address for that device
+ *    (with that device current); make it before any stream capture.
+ *  - All calls share the array: a scale-fixing first append clears it before
+ *    use; calls whose work overlaps on the GPU race on it, so serialise them. */
+NVKV_API nvkv_status nvfp4_kv_append_noalloc(const nvkv_desc *desc, const nvkv_cache *cache,
+                                             nvkv_ring *ring, const void *k, const void *v,
+                                             nvkv_stream stream);
+
 /* The bf16-KV twin: same slot logic, the chunk's bf16 K/V copied as is. */
 NVKV_API nvkv_status bf16_kv_append(const nvkv_desc *desc, const nvkv_cache *cache, nvkv_ring *ring,
                            const void *k, const void *v, nvkv_stream stream);

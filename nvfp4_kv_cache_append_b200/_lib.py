@@ -88,6 +88,7 @@ def _load():
         "nvkv_ring_push_chunk": (i32, [D, R, i32p]),
         "nvfp4_kv_append": (i32, [D, C, R, vp, vp, vp]),
         "bf16_kv_append": (i32, [D, C, R, vp, vp, vp]),
+        "nvfp4_kv_append_noalloc": (i32, [D, C, R, vp, vp, vp]),
         "nvkv_attention_workspace_bytes": (sz, [D]),
         "chunk_attention_nvfp4kv": (i32, [D, C, R, vp, vp, vp, vp, sz, vp]),
         "chunk_attention_bf16kv": (i32, [D, C, R, vp, vp, vp, vp, sz, vp]),
@@ -168,6 +169,12 @@ def nvkv_ring_push_chunk(desc: nvkv_desc, ring: nvkv_ring):
 def nvfp4_kv_append(desc, cache, ring, k_ptr, v_ptr, stream=0) -> None:
     _check(lib.nvfp4_kv_append(ctypes.byref(desc), ctypes.byref(cache), ctypes.byref(ring),
                                k_ptr, v_ptr, stream), "nvfp4_kv_append")
+
+
+def nvfp4_kv_append_noalloc(desc, cache, ring, k_ptr, v_ptr, stream=0) -> None:
+    _check(lib.nvfp4_kv_append_noalloc(ctypes.byref(desc), ctypes.byref(cache),
+                                       ctypes.byref(ring), k_ptr, v_ptr, stream),
+           "nvfp4_kv_append_noalloc")
 
 
 def bf16_kv_append(desc, cache, ring, k_ptr, v_ptr, stream=0) -> None:
