@@ -246,7 +246,9 @@ NVKV_API size_t nvkv_attention_workspace_bytes(const nvkv_desc *desc);
  * chunk included, in full).  Keys are read from the cache, dequantized and
  * rotated by 3D RoPE at (their frame's RoPE index, h, w); queries are rotated
  * at (the RoPE index of their own frame, h, w).  Logits use 1/sqrt(128).
- * NVKV_ERR_STATE if nothing was appended yet. */
+ * NVKV_ERR_STATE if nothing was appended yet; NVKV_ERR_UNSUPPORTED for a RoPE
+ * split other than 44/42/42, grid_h or grid_w above 256, or (NVFP4) an odd
+ * number of tokens per frame. */
 NVKV_API nvkv_status chunk_attention_nvfp4kv(const nvkv_desc *desc, const nvkv_cache *cache,
                                     const nvkv_ring *ring, const void *q, void *out, float *lse,
                                     void *workspace, size_t workspace_bytes, nvkv_stream stream);

@@ -183,9 +183,14 @@ nvkv_status attention_common(const nvkv_desc *desc, const nvkv_cache *cache,
     a.grid_w = desc->grid_w;
     a.kv_dtype = dtype;
     a.grid_h = desc->grid_h;
-    // the attention kernels are built for the 44/42/42 split and small grids
+    a.inv_T = 1.0f / (float)a.T;
+    a.inv_grid_w = 1.0f / (float)desc->grid_w;
+    // the attention kernels are built for the 44/42/42 split and small grids;
+    // the NVFP4 kernel stages scale rows with 16-byte bulk copies, which needs
+    // an even number of tokens per frame
     if (desc->rope_split[0] != 44 || desc->rope_split[1] != 42 || desc->rope_split[2] != 42 ||
-        desc->grid_h > 256 || desc->grid_w > 256)
+        desc->grid_h > 256 || desc->grid_w > 256 ||
+        (dtype == NVKV_KV_NVFP4 && ((desc->grid_h * desc->grid_w) & 1)))
         return NVKV_ERR_UNSUPPORTED;
     {
         int p = 0;

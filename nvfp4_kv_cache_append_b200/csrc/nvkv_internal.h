@@ -47,6 +47,7 @@ struct AttnLaunch {
     int q_pos0[NVKV_MAX_BATCH];      // RoPE frame index of the chunk's first frame
     VisFrame vis[NVKV_MAX_BATCH][NVKV_MAX_FRAMES];
     int grid_h;
+    float inv_T, inv_grid_w;         // 1/T and 1/grid_w (division by reciprocal + fix-up)
     int n_fpos;                      // frame positions used: 0 .. n_fpos-1
     float theta[64];                 // RoPE angle per unit position of each channel pair
 };
