@@ -236,7 +236,12 @@ NVKV_API nvkv_status nvfp4_kv_append_noalloc(const nvkv_desc *desc, const nvkv_c
 NVKV_API nvkv_status bf16_kv_append(const nvkv_desc *desc, const nvkv_cache *cache, nvkv_ring *ring,
                            const void *k, const void *v, nvkv_stream stream);
 
-/* Device workspace the attention calls need (may be 0). */
+/* Device workspace the attention calls need on the current device (0 for an
+ * invalid desc or without a device).  The attention kernels run a persistent
+ * grid of CTA pairs; query tiles cut between pairs leave partial results
+ * here and the last pair to finish merges them.  The caller allocates it once,
+ * 16-byte aligned, and zero-fills it before first use; every call leaves it
+ * zeroed again.  Calls sharing a workspace must not overlap on the GPU. */
 NVKV_API size_t nvkv_attention_workspace_bytes(const nvkv_desc *desc);
 
 /* Block-causal chunk attention of the newest chunk.  q: device bf16
@@ -246,7 +251,9 @@ NVKV_API size_t nvkv_attention_workspace_bytes(const nvkv_desc *desc);
  * chunk included, in full).  Keys are read from the cache, dequantized and
  * rotated by 3D RoPE at (their frame's RoPE index, h, w); queries are rotated
  * at (the RoPE index of their own frame, h, w).  Logits use 1/sqrt(128).
- * NVKV_ERR_STATE if nothing was appended yet; NVKV_ERR_UNSUPPORTED for a RoPE
+ * workspace: device memory of nvkv_attention_workspace_bytes() bytes (else
+ * NVKV_ERR_CAPACITY).  NVKV_ERR_STATE if nothing was appended yet;
+ * NVKV_ERR_UNSUPPORTED for a RoPE
  * split other than 44/42/42, grid_h or grid_w above 256, or (NVFP4) an odd
  * number of tokens per frame. */
 NVKV_API nvkv_status chunk_attention_nvfp4kv(const nvkv_desc *desc, const nvkv_cache *cache,

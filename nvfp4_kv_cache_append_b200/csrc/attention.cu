@@ -11,33 +11,36 @@
 // video generation", section "NVFP4, sequence parallel and the async decode
 // path": FP4 KV dequantization and fused RoPE).
 //
-// Structure: one CTA per (256 query rows = Q tiles A and B, head, batch);
-// key tiles of 64; 16 warps.
-//   warps 0-3    softmax of Q tile A, warps 4-7 softmax of Q tile B: thread r
-//                owns query row r = TMEM lane r.  Per key tile it reads its 64
-//                logits once from TMEM, keeps the online softmax in registers
-//                (lazy rescale of O when the row max grows by more than 2^8)
-//                and writes P (f16) back into TMEM over S.
-//   warps 8-11   K converters: first RoPE-rotate Q_A/Q_B into TMEM; then per
-//                key tile two threads per key, each half a row: E2M1 codes ->
-//                f16 by cvt, times the E4M3 block scale (exact in f16), RoPE in
-//                packed f16x2 math, into a 128-byte-swizzled K-major UMMA tile.
-//   warps 12-13  V converters: one thread per key: decode and scale into the
-//                V tile (read by the MMA as MN-major).
-//   warp 14      producer: bulk async copies (TMA engine) of each tile's packed
-//                code and scale rows, run by run, into a 4-stage staging ring.
-//   warp 15      TMEM allocation and the MMA issuer (one thread):
-//                S = Q K^T (Q from TMEM, K from shared memory) and O += P V
-//                (P from TMEM, V from shared memory), kind::f16, f32
-//                accumulators.  TMEM: Q_A | Q_B | S_A | S_B | O_A | O_B
-//                (64+64+64+64+128+128 = 512 columns).  Issue order per tile:
-//                PV(A) S'(A) PV(B) S'(B), so one softmax group always has work.
-// K and V tiles are double buffered; with Q and P in TMEM the tensor core only
-// reads K and V from shared memory.
-// The global scales are folded out of the dequantization: s_g(K) goes into the
-// softmax scale, s_g(V) into the epilogue.  Both caches compute with f16
-// operands (dequantized NVFP4 values are exact there).
-// Every mbarrier wait is bounded; on expiry the CTA records NVKV_ERR_TIMEOUT
+// Structure.  A cluster of two CTAs (one per SM) owns a pair of 128-row query
+// tiles of one (b, h) at a time; key tiles are 128 keys.  Every MMA is a
+// pair MMA (tcgen05 cta_group::2, M = 256) issued by the even CTA: each SM
+// computes its own 128 rows and holds half of each B operand, so each SM
+// dequantizes only half of every key tile:
+//   K: keys [64r, 64r+64) of the tile (all 128 channels),
+//   V: channels [64r, 64r+64) of all 128 keys   (r = CTA rank in the pair).
+// Per CTA, 16 warps:
+//   warps 0-3    softmax: thread r owns query row r = TMEM lane r.  Per tile a
+//                max pass and a probability pass over the 128 logits in TMEM,
+//                P (f16) written back over S; online softmax with lazy rescale
+//                of O (when the row max grows by more than 2^8).
+//   warps 4-7    K converters (two threads per key) and, per work segment,
+//                the RoPE-rotated Q tile into TMEM.
+//   warps 8-11   V converters (one thread per key).
+//   warp 12      producer: bulk async copies (TMA engine) of the packed code
+//                and scale rows into a 4-stage staging ring (NVFP4 only).
+//   warp 13      TMEM allocation (both CTAs) and, in the even CTA, the MMA
+//                issuer: S = Q K^T into one of two S buffers while the softmax
+//                reads the other, then O += P V.
+// TMEM per CTA: Q (64 cols, f16 pairs) | S0 (128) | S1 (128) | O (128).
+// Dequantized values are exact in f16 (E2M1 code x E4M3 scale); the global
+// scales fold into the softmax scale (K) and the epilogue (V).
+//
+// Scheduling: the grid is persistent (one CTA pair per slot).  The (b, h,
+// pair) work items are laid end to end in tiles and cut into equal
+// contiguous ranges, one per slot; an item cut by a range boundary is
+// finished by several slots, which leave partial (O, max, sum) records in the
+// workspace and the last one to finish merges them.
+// Every mbarrier wait is bounded; on expiry the pair records NVKV_ERR_TIMEOUT
 // in the status word, unwinds, waits for its own MMAs and frees TMEM.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -47,6 +50,78 @@
 
 namespace nvkv {
 namespace {
+
+constexpr int BM = 128;                // query rows per CTA (the pair covers 256)
+constexpr int BN = 128;                // keys per tile
+constexpr int NTHREADS = 512;
+constexpr int NSTAGE = 4;              // staging ring depth
+constexpr int MAX_SEG = 96;            // work segments per slot
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s per wait
+constexpr int PAIRS_F = 22, PAIRS_H = 21, PAIRS_W = 21;   // 44 / 42 / 42 channels
+
+constexpr uint32_t K_TILE = 16384;      // 64 keys x 128 ch f16, K-major, 128-B swizzle
+constexpr uint32_t K_HALF = 8192;       // one 64-channel half of it
+constexpr uint32_t V_TILE = 16384;      // 128 keys x 64 ch f16, MN-major, 128-B swizzle
+constexpr uint32_t OFF_K = 0;                         // two buffers
+constexpr uint32_t OFF_V = OFF_K + 2 * K_TILE;        // two buffers
+constexpr uint32_t OFF_STG = OFF_V + 2 * V_TILE;      // staging ring
+constexpr uint32_t STG_KC = 0, STG_KS = 4096, STG_VC = 4608, STG_VS = 12800;
+constexpr uint32_t STG_BYTES = 13824;
+constexpr uint32_t OFF_TAB = OFF_STG + NSTAGE * STG_BYTES;   // RoPE tables
+
+// TMEM columns
+constexpr uint32_t TM_Q = 0;      // f16 pairs of the 128 channels
+constexpr uint32_t TM_S = 64;     // S buffers at 64 and 192 (f32); P over S
+constexpr uint32_t TM_O = 320;    // f32
+
+constexpr int PART_FLOATS = 130;  // O (128) + max + sum per row of a partial record
+
+enum Bar {
+    B_QREADY = 0,                         // [even CTA] both Q tiles in TMEM (256)
+    B_KFULL = 1,                          // [even] + buffer: K halves (256)
+    B_VFULL = 3,                          // [even] + buffer: V halves (256)
+    B_P = 5,                              // [even] + buffer: P of both tiles (256)
+    B_OFREE = 7,                          // [even] epilogues read O (256)
+    B_S = 8,                              // + buffer: S written (commit)
+    B_KFREE = 10,                         // + buffer (commit)
+    B_VFREE = 12,                         // + buffer (commit)
+    B_QFREE = 14,                         // segment's last S done (commit)
+    B_ODONE = 15,                         // segment's last PV done (commit)
+    B_MMADONE = 16,                       // everything issued is done (commit)
+    B_STG_FULL = 17,                      // + stage (producer, 1 + bytes)
+    B_STG_EMPTY = B_STG_FULL + NSTAGE,    // + stage (K and V converters, 256)
+    N_BARS = B_STG_EMPTY + NSTAGE
+};
+
+struct Segment {
+    int b, h, p;        // work item: batch, head, query tile pair
+    int t0, t1;         // key tiles [t0, t1) of the item
+    int n_chunks;       // slots sharing the item (1: this segment finishes it)
+    int part;           // partial record index of this segment
+    int first_slot;     // slot holding the item's first chunk (counter index)
+    int item_start;     // flattened tile index of the item's tile 0
+};
+
+struct SharedCtl {
+    uint64_t bar[N_BARS];
+    int abort;
+    uint32_t tmem_base;
+    int n_seg;
+    int merge_flag;
+    Segment seg[MAX_SEG];
+};
+
+// byte offset of 16-byte chunk c (0..15) of key row r (0..63) in a K tile
+__device__ __forceinline__ uint32_t swz_k(int r, int c)
+{
+    return (uint32_t)((c >> 3) * K_HALF + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+// byte offset of 16-byte chunk c (0..7, channels 8c..8c+7) of key k in a V tile
+__device__ __forceinline__ uint32_t swz_v(int k, int c)
+{
+    return (uint32_t)(k * 128 + ((c ^ (k & 7)) << 4));
+}
 
 __device__ __forceinline__ float ex2(float x)
 {
@@ -72,10 +147,26 @@ __device__ __forceinline__ void sts16(uint32_t addr, uint32_t a, uint32_t b, uin
                  : "memory");
 }
 
+__device__ __forceinline__ uint4 lds16(uint32_t addr)
+{
+    uint4 r;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "r"(addr));
+    return r;
+}
+
 __device__ __forceinline__ uint2 lds8(uint32_t addr)
 {
     uint2 r;
     asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(addr));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t lds4(uint32_t addr)
+{
+    uint32_t r;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(addr));
     return r;
 }
 
@@ -114,71 +205,6 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi)
     return as_u(__floats2half2_rn(lo, hi));
 }
 
-constexpr int BM = 128;                // rows of one Q tile; a CTA holds two
-constexpr int BN = 64;                 // keys per tile
-constexpr int NTHREADS = 512;
-constexpr int NSTAGE = 4;              // staging ring depth
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s per wait
-constexpr int PAIRS_F = 22, PAIRS_H = 21, PAIRS_W = 21;   // 44 / 42 / 42 channels
-
-constexpr uint32_t KV_TILE = 16384;     // 64 keys x 128 x f16
-constexpr uint32_t KV_HALF = 8192;      // one 64-element half of a K/V tile
-constexpr uint32_t OFF_K = 0;                         // two buffers
-constexpr uint32_t OFF_V = OFF_K + 2 * KV_TILE;       // two buffers
-constexpr uint32_t OFF_STG = OFF_V + 2 * KV_TILE;     // staging ring
-constexpr uint32_t STG_KC = 0, STG_VC = 4096, STG_KS = 8192, STG_VS = 8704;
-constexpr uint32_t STG_BYTES = 9216;
-constexpr uint32_t OFF_TAB = OFF_STG + NSTAGE * STG_BYTES;   // RoPE tables
-
-// TMEM columns
-constexpr uint32_t TM_Q = 0;      // Q_A, Q_B: 64 columns each (f16 pairs)
-constexpr uint32_t TM_S = 128;    // S_A, S_B: 64 columns each (f32); P over S
-constexpr uint32_t TM_O = 256;    // O_A, O_B: 128 columns each (f32)
-
-enum Bar {
-    B_Q = 0,
-    B_STG_FULL = 1,                    // + stage
-    B_STG_EMPTY = B_STG_FULL + NSTAGE, // + stage
-    B_KFULL = B_STG_EMPTY + NSTAGE,    // + buffer
-    B_KFREE = B_KFULL + 2,             // + buffer
-    B_VFULL = B_KFREE + 2,             // + buffer
-    B_VFREE = B_VFULL + 2,             // + buffer
-    B_S = B_VFREE + 2,                 // + Q tile: S of that tile written
-    B_P = B_S + 2,                     // + Q tile: P of that tile written
-    B_ODONE = B_P + 2,
-    B_MMADONE = B_ODONE + 1,
-    N_BARS = B_MMADONE + 1
-};
-
-struct SharedCtl {
-    uint64_t bar[N_BARS];
-    int abort;
-    uint32_t tmem_base;
-};
-
-// byte offset of 16-byte chunk c (0..15) of row r inside a 64-row K-major
-// operand tile with 128-byte swizzle: two 64-element halves of 8 KB.
-__device__ __forceinline__ uint32_t swz(int r, int c)
-{
-    return (uint32_t)((c >> 3) * KV_HALF + r * 128 + (((c & 7) ^ (r & 7)) << 4));
-}
-
-__device__ __forceinline__ uint4 lds16(uint32_t addr)
-{
-    uint4 r;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "r"(addr));
-    return r;
-}
-
-__device__ __forceinline__ uint32_t lds4(uint32_t addr)
-{
-    uint32_t r;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(addr));
-    return r;
-}
-
 // x / d for 0 <= x < 2^24 by a float reciprocal with a one-step fix-up
 __device__ __forceinline__ int div_fast(int x, int d, float inv)
 {
@@ -192,15 +218,28 @@ struct Ctx {
     const AttnLaunch *a;
     uint8_t *smem;
     SharedCtl *ctl;
-    int b, h, q0, n_keys, n_tiles;
     uint32_t sbase;                 // shared-space address of smem
     uint32_t tab_f, tab_h, tab_w;   // byte offsets of the three RoPE tables
+    uint32_t rank;                  // CTA rank in the pair
+    uint32_t lead_bar;              // shared::cluster address of the even CTA's bar[0]
+    uint32_t peer_abort;            // shared::cluster address of the other CTA's abort flag
+    int slot;
 };
+
+__device__ __forceinline__ uint32_t lead(const Ctx &c, int bar) { return c.lead_bar + bar * 8; }
+
+__device__ __forceinline__ void set_abort(Ctx &c)
+{
+    if (atomicExch(&c.ctl->abort, 1) == 0) {
+        atomicCAS(c.a->status, 0, (int)NVKV_ERR_TIMEOUT);
+        ptx::st_cluster_u32(c.peer_abort, 1u);
+    }
+}
 
 __device__ __forceinline__ bool wait(Ctx &c, int bar, uint32_t parity)
 {
-    if (ptx::mbar_wait(&c.ctl->bar[bar], parity, &c.ctl->abort, WAIT_LIMIT_NS)) return true;
-    if (atomicExch(&c.ctl->abort, 1) == 0) atomicCAS(c.a->status, 0, (int)NVKV_ERR_TIMEOUT);
+    if (ptx::mbar_wait_cluster(&c.ctl->bar[bar], parity, &c.ctl->abort, WAIT_LIMIT_NS)) return true;
+    set_abort(c);
     return false;
 }
 
@@ -210,6 +249,67 @@ __device__ __forceinline__ bool wait_warp(Ctx &c, int bar, uint32_t parity)
 {
     const bool ok = wait(c, bar, parity);
     return __all_sync(0xFFFFFFFFu, ok);
+}
+
+// ------------------------------------------------------------ schedule
+
+__device__ __forceinline__ int key_tiles(const AttnLaunch &a, int b)
+{
+    return (a.n_vis[b] * a.T + BN - 1) / BN;
+}
+
+__device__ __forceinline__ long long total_tiles(const AttnLaunch &a)
+{
+    long long total = 0;
+    for (int b = 0; b < a.B; ++b) total += (long long)a.H * a.n_pairs * key_tiles(a, b);
+    return total;
+}
+
+// Segments of this slot: the items (b, h, p) in order, each n_kt(b) tiles,
+// laid end to end and cut into n_slots equal ranges.
+__device__ void build_schedule(Ctx &c)
+{
+    const AttnLaunch &a = *c.a;
+    const long long total = total_tiles(a);
+    const long long target = (total + a.n_slots - 1) / a.n_slots;
+    const long long beg = (long long)c.slot * target;
+    const long long end = min(total, beg + target);
+    int n = 0;
+    long long u = beg;
+    long long base = 0;
+    for (int b = 0; b < a.B && u < end; ++b) {
+        const int nkt = key_tiles(a, b);
+        const long long span = (long long)a.H * a.n_pairs * nkt;
+        while (u < end && u < base + span && n < MAX_SEG) {
+            const long long off = u - base;
+            const int item = (int)(off / nkt);
+            const int t0 = (int)(off - (long long)item * nkt);
+            const long long item_start = base + (long long)item * nkt;
+            const long long seg_end = min(end, item_start + nkt);
+            Segment &s = c.ctl->seg[n++];
+            s.b = b;
+            s.h = item / a.n_pairs;
+            s.p = item - s.h * a.n_pairs;
+            s.t0 = t0;
+            s.t1 = t0 + (int)(seg_end - u);
+            const int first = (int)(item_start / target);
+            const int last = (int)((item_start + nkt - 1) / target);
+            s.n_chunks = last - first + 1;
+            s.first_slot = first;
+            s.item_start = (int)item_start;
+            s.part = 2 * c.slot + (u == beg ? 0 : 1);
+            u = seg_end;
+        }
+        base += span;
+    }
+    c.ctl->n_seg = n;
+}
+
+// partial record index of chunk k of an item (see build_schedule)
+__device__ __forceinline__ int chunk_part(const Segment &s, int k, long long target)
+{
+    const int slot = s.first_slot + k;
+    return 2 * slot + ((k == 0 && (long long)s.item_start > (long long)slot * target) ? 1 : 0);
 }
 
 // ------------------------------------------------------------ RoPE tables
@@ -274,18 +374,18 @@ struct KeyPos {
     size_t grow;   // global row index into the [B][H][R] planes
 };
 
-__device__ __forceinline__ KeyPos key_pos(const Ctx &c, int key)
+__device__ __forceinline__ KeyPos key_pos(const Ctx &c, int b, int h, int n_keys, int key)
 {
     const AttnLaunch &a = *c.a;
     KeyPos k;
-    k.valid = key < c.n_keys;
+    k.valid = key < n_keys;
     const int kk = k.valid ? key : 0;
     const int f = div_fast(kk, a.T, a.inv_T);
     const int tok = kk - f * a.T;
-    const VisFrame vf = a.vis[c.b][f];
+    const VisFrame vf = a.vis[b][f];
     const int hp = div_fast(tok, a.grid_w, a.inv_grid_w);
     k.rr = rope_rows(c, vf.rope_pos, hp, tok - hp * a.grid_w);
-    k.grow = (size_t)(c.b * a.H + c.h) * a.R + (size_t)vf.slot * a.T + tok;
+    k.grow = (size_t)(b * a.H + h) * a.R + (size_t)vf.slot * a.T + tok;
     return k;
 }
 
@@ -294,16 +394,16 @@ __device__ __forceinline__ KeyPos key_pos(const Ctx &c, int key)
 // Q row `row` of the chunk -> RoPE in f32 -> f16 pairs in TMEM columns
 // [tcol, tcol + 64) of this thread's lane.
 template <bool FP4>
-__device__ void load_q_tmem(const Ctx &c, int row, uint32_t tcol)
+__device__ void load_q_tmem(const Ctx &c, int b, int h, int row, uint32_t tcol)
 {
     const AttnLaunch &a = *c.a;
     const bool valid = row < a.Lq;
     const uint4 *src = reinterpret_cast<const uint4 *>(a.q) +
-                       (((size_t)c.b * a.Lq + (valid ? row : 0)) * a.H + c.h) * 16;
+                       (((size_t)b * a.Lq + (valid ? row : 0)) * a.H + h) * 16;
     const int frame = valid ? div_fast(row, a.T, a.inv_T) : 0;
     const int tok = valid ? row - frame * a.T : 0;
     const int hp = div_fast(tok, a.grid_w, a.inv_grid_w);
-    const RopeRows rr = rope_rows(c, a.q_pos0[c.b] + frame, hp, tok - hp * a.grid_w);
+    const RopeRows rr = rope_rows(c, a.q_pos0[b] + frame, hp, tok - hp * a.grid_w);
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
         uint32_t o[32];
@@ -334,18 +434,18 @@ __device__ void load_q_tmem(const Ctx &c, int row, uint32_t tcol)
 
 // ------------------------------------------------------------ converters
 
-// K, NVFP4: key row r, half HH (channel pairs 32HH .. 32HH+31) from the
-// staging stage into the K tile: decode, scale (exact), rotate.  An invalid
-// row reads zero codes and writes zeros.
+// K, NVFP4: staging key row sr (0..63), channel half HH (pairs 32HH ..
+// 32HH+31) into row sr of the K tile: decode, scale (exact), rotate.  An
+// invalid key reads zero codes and writes zeros.
 template <int HH>
-__device__ __forceinline__ void conv_k_fp4(uint32_t stg, int r, const KeyPos &k, uint32_t kdst)
+__device__ __forceinline__ void conv_k_fp4(uint32_t stg, int sr, const KeyPos &k, uint32_t kdst)
 {
     uint4 w0 = make_uint4(0, 0, 0, 0), w1 = w0;
     uint32_t sc = 0;
     if (k.valid) {
-        w0 = lds16(stg + STG_KC + r * 64 + HH * 32);
-        w1 = lds16(stg + STG_KC + r * 64 + HH * 32 + 16);
-        sc = lds4(stg + STG_KS + r * 8 + HH * 4);
+        w0 = lds16(stg + STG_KC + sr * 64 + HH * 32);
+        w1 = lds16(stg + STG_KC + sr * 64 + HH * 32 + 16);
+        sc = lds4(stg + STG_KS + sr * 8 + HH * 4);
     }
     const uint32_t code[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
@@ -361,36 +461,37 @@ __device__ __forceinline__ void conv_k_fp4(uint32_t stg, int r, const KeyPos &k,
             // (x c - y s, y c + x s)
             o[q] = as_u(__hfma2(__lowhigh2highlow(v), as_h2(e.y), __hmul2(v, as_h2(e.x))));
         }
-        sts16(kdst + swz(r, HH * 8 + cc), o[0], o[1], o[2], o[3]);
+        sts16(kdst + swz_k(sr, HH * 8 + cc), o[0], o[1], o[2], o[3]);
     }
 }
 
-// V, NVFP4: one key row: decode and scale.
-__device__ __forceinline__ void conv_v_fp4(uint32_t stg, int r, bool valid, uint32_t vdst)
+// V, NVFP4: staging key row k (0..127), this CTA's channel half (bytes
+// [32 half, 32 half + 32) of the packed row, scale blocks 4 half .. +3).
+__device__ __forceinline__ void conv_v_fp4(uint32_t stg, int k, int half, bool valid,
+                                           uint32_t vdst)
 {
-    uint2 sc = make_uint2(0, 0);
-    if (valid) sc = lds8(stg + STG_VS + r * 8);
+    uint4 w0 = make_uint4(0, 0, 0, 0), w1 = w0;
+    uint32_t sc = 0;
+    if (valid) {
+        w0 = lds16(stg + STG_VC + k * 64 + half * 32);
+        w1 = lds16(stg + STG_VC + k * 64 + half * 32 + 16);
+        sc = lds4(stg + STG_VS + k * 8 + half * 4);
+    }
+    const uint32_t code[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-    for (int g = 0; g < 4; ++g) {
-        const uint4 w = valid ? lds16(stg + STG_VC + r * 64 + g * 16) : make_uint4(0, 0, 0, 0);
-        const uint32_t code[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int cc4 = 0; cc4 < 4; ++cc4) {
-            const int cc = g * 4 + cc4;                 // output chunk, block cc / 2
-            const uint32_t sword = (cc >> 1) < 4 ? sc.x : sc.y;
-            const __half2 sb = e4m3_to_h2((sword >> (8 * ((cc >> 1) & 3))) & 0xFFu);
-            uint32_t hq[4];
-            e2m1x8_to_f16(code[cc4], hq);
-            sts16(vdst + swz(r, cc), as_u(__hmul2(as_h2(hq[0]), sb)),
-                  as_u(__hmul2(as_h2(hq[1]), sb)), as_u(__hmul2(as_h2(hq[2]), sb)),
-                  as_u(__hmul2(as_h2(hq[3]), sb)));
-        }
+    for (int cc = 0; cc < 8; ++cc) {          // channels 8cc .. 8cc+7 of the half
+        const __half2 sb = e4m3_to_h2((sc >> (8 * (cc >> 1))) & 0xFFu);
+        uint32_t hq[4];
+        e2m1x8_to_f16(code[cc], hq);
+        sts16(vdst + swz_v(k, cc), as_u(__hmul2(as_h2(hq[0]), sb)),
+              as_u(__hmul2(as_h2(hq[1]), sb)), as_u(__hmul2(as_h2(hq[2]), sb)),
+              as_u(__hmul2(as_h2(hq[3]), sb)));
     }
 }
 
-// K, bf16 twin: key row r, half HH, read from global memory, RoPE in f32.
+// K, bf16 twin: channel half HH of key k from global memory, RoPE in f32.
 template <int HH>
-__device__ __forceinline__ void conv_k_bf16(const Ctx &c, int r, const KeyPos &k, uint32_t kdst)
+__device__ __forceinline__ void conv_k_bf16(const Ctx &c, int sr, const KeyPos &k, uint32_t kdst)
 {
     const uint4 *src = reinterpret_cast<const uint4 *>(c.a->k_data) + k.grow * 16 + HH * 8;
 #pragma unroll
@@ -406,114 +507,142 @@ __device__ __forceinline__ void conv_k_bf16(const Ctx &c, int r, const KeyPos &k
             const float cs = __uint_as_float(e.x), sn = __uint_as_float(e.y);
             o[q] = pack_f16(x * cs - y * sn, x * sn + y * cs);
         }
-        sts16(kdst + swz(r, HH * 8 + cc), o[0], o[1], o[2], o[3]);
+        sts16(kdst + swz_k(sr, HH * 8 + cc), o[0], o[1], o[2], o[3]);
     }
 }
 
-// V, bf16 twin: one key row from global memory, converted to f16.
-__device__ __forceinline__ void conv_v_bf16(const Ctx &c, int r, const KeyPos &k, uint32_t vdst)
+// V, bf16 twin: this CTA's channel half of key k from global memory.
+__device__ __forceinline__ void conv_v_bf16(const Ctx &c, int kk, int half, const KeyPos &k,
+                                            uint32_t vdst)
 {
-    const uint4 *src = reinterpret_cast<const uint4 *>(c.a->v_data) + k.grow * 16;
-#pragma unroll 4
-    for (int cc = 0; cc < 16; ++cc) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(c.a->v_data) + k.grow * 16 + half * 8;
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
         const uint4 w = k.valid ? ldg16(src + cc) : make_uint4(0, 0, 0, 0);
         const uint32_t u[4] = {w.x, w.y, w.z, w.w};
         uint32_t o[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q)
             o[q] = pack_f16(__uint_as_float(u[q] << 16), __uint_as_float(u[q] & 0xFFFF0000u));
-        sts16(vdst + swz(r, cc), o[0], o[1], o[2], o[3]);
+        sts16(vdst + swz_v(kk, cc), o[0], o[1], o[2], o[3]);
     }
 }
 
-// warps 8-11: Q prologue, then K tiles (thread t: key t & 63, half t >> 6)
+// warps 4-7: per segment the Q tile into TMEM, then K halves of the tiles
 template <bool FP4>
 __device__ void k_converter_role(Ctx &c)
 {
-    const int t = threadIdx.x - 256;          // 0..127, TMEM lane t
+    const AttnLaunch &a = *c.a;
+    const int t = threadIdx.x - 128;          // 0..127, TMEM lane t
     const uint32_t lane_off = (uint32_t)(t & ~31) << 16;
     const uint32_t tmem = c.ctl->tmem_base;
-    load_q_tmem<FP4>(c, c.q0 + t, tmem + lane_off + TM_Q);
-    load_q_tmem<FP4>(c, c.q0 + BM + t, tmem + lane_off + TM_Q + 64);
-    ptx::tmem_wait_st();
-    ptx::tc_fence_before();
-    ptx::mbar_arrive(&c.ctl->bar[B_Q]);
-
-    const int r = t & 63, hh = t >> 6;        // hh is warp-uniform
-    for (int j = 0; j < c.n_tiles; ++j) {
-        const int s = j % NSTAGE, kb = j & 1;
-        const uint32_t stg = c.sbase + OFF_STG + s * STG_BYTES;
-        const uint32_t kdst = c.sbase + OFF_K + kb * KV_TILE;
-        const KeyPos k = key_pos(c, j * BN + r);
-        if (FP4 && !wait(c, B_STG_FULL + s, (j / NSTAGE) & 1)) return;
-        if (j >= 2 && !wait(c, B_KFREE + kb, ((j - 2) >> 1) & 1)) return;
-        if (FP4) {
-            if (hh == 0) conv_k_fp4<0>(stg, r, k, kdst);
-            else conv_k_fp4<1>(stg, r, k, kdst);
-        } else {
-            if (hh == 0) conv_k_bf16<0>(c, r, k, kdst);
-            else conv_k_bf16<1>(c, r, k, kdst);
+    const int sr = t & 63, hh = t >> 6;       // staging key row, channel half (warp-uniform)
+    int g = 0;                                 // tiles processed by this CTA
+    for (int si = 0; si < c.ctl->n_seg; ++si) {
+        const Segment sg = c.ctl->seg[si];
+        const int n_keys = a.n_vis[sg.b] * a.T;
+        if (si > 0 && !wait_warp(c, B_QFREE, (si - 1) & 1)) return;
+        ptx::tc_fence_after();
+        load_q_tmem<FP4>(c, sg.b, sg.h, (2 * sg.p + (int)c.rank) * BM + t, tmem + lane_off + TM_Q);
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive_remote(lead(c, B_QREADY));
+        for (int tile = sg.t0; tile < sg.t1; ++tile, ++g) {
+            const int s = g % NSTAGE, kb = g & 1;
+            const uint32_t stg = c.sbase + OFF_STG + s * STG_BYTES;
+            const uint32_t kdst = c.sbase + OFF_K + kb * K_TILE;
+            const KeyPos k = key_pos(c, sg.b, sg.h, n_keys, tile * BN + 64 * (int)c.rank + sr);
+            if (FP4 && !wait(c, B_STG_FULL + s, (g / NSTAGE) & 1)) return;
+            if (g >= 2 && !wait(c, B_KFREE + kb, ((g - 2) >> 1) & 1)) return;
+            if (FP4) {
+                if (hh == 0) conv_k_fp4<0>(stg, sr, k, kdst);
+                else conv_k_fp4<1>(stg, sr, k, kdst);
+            } else {
+                if (hh == 0) conv_k_bf16<0>(c, sr, k, kdst);
+                else conv_k_bf16<1>(c, sr, k, kdst);
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::mbar_arrive_remote(lead(c, B_KFULL + kb));
+            if (FP4) ptx::mbar_arrive(&c.ctl->bar[B_STG_EMPTY + s]);
         }
-        ptx::fence_proxy_async_smem();
-        ptx::mbar_arrive(&c.ctl->bar[B_KFULL + kb]);
-        if (FP4) ptx::mbar_arrive(&c.ctl->bar[B_STG_EMPTY + s]);
     }
 }
 
-// warps 12-13: V tiles (thread t: key t)
+// warps 8-11: this CTA's channel half of V for all 128 keys of each tile
 template <bool FP4>
 __device__ void v_converter_role(Ctx &c)
 {
-    const int r = threadIdx.x - 384;          // 0..63
-    for (int j = 0; j < c.n_tiles; ++j) {
-        const int s = j % NSTAGE, vb = j & 1;
-        const uint32_t stg = c.sbase + OFF_STG + s * STG_BYTES;
-        const uint32_t vdst = c.sbase + OFF_V + vb * KV_TILE;
-        if (FP4 && !wait(c, B_STG_FULL + s, (j / NSTAGE) & 1)) return;
-        if (j >= 2 && !wait(c, B_VFREE + vb, ((j - 2) >> 1) & 1)) return;
-        if (FP4) {
-            conv_v_fp4(stg, r, j * BN + r < c.n_keys, vdst);
-        } else {
-            const KeyPos k = key_pos(c, j * BN + r);
-            conv_v_bf16(c, r, k, vdst);
+    const AttnLaunch &a = *c.a;
+    const int k = threadIdx.x - 256;          // key of the tile, 0..127
+    int g = 0;
+    for (int si = 0; si < c.ctl->n_seg; ++si) {
+        const Segment sg = c.ctl->seg[si];
+        const int n_keys = a.n_vis[sg.b] * a.T;
+        for (int tile = sg.t0; tile < sg.t1; ++tile, ++g) {
+            const int s = g % NSTAGE, vb = g & 1;
+            const uint32_t stg = c.sbase + OFF_STG + s * STG_BYTES;
+            const uint32_t vdst = c.sbase + OFF_V + vb * V_TILE;
+            if (FP4 && !wait(c, B_STG_FULL + s, (g / NSTAGE) & 1)) return;
+            if (g >= 2 && !wait(c, B_VFREE + vb, ((g - 2) >> 1) & 1)) return;
+            if (FP4) {
+                conv_v_fp4(stg, k, (int)c.rank, tile * BN + k < n_keys, vdst);
+            } else {
+                const KeyPos kp = key_pos(c, sg.b, sg.h, n_keys, tile * BN + k);
+                conv_v_bf16(c, k, (int)c.rank, kp, vdst);
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::mbar_arrive_remote(lead(c, B_VFULL + vb));
+            if (FP4) ptx::mbar_arrive(&c.ctl->bar[B_STG_EMPTY + s]);
         }
-        ptx::fence_proxy_async_smem();
-        ptx::mbar_arrive(&c.ctl->bar[B_VFULL + vb]);
-        if (FP4) ptx::mbar_arrive(&c.ctl->bar[B_STG_EMPTY + s]);
     }
 }
 
 // ------------------------------------------------------------ producer
 
-// Bulk copies of tile j's packed rows: every run of consecutive keys that
-// lies in one frame is contiguous in the planes.  Run starts and lengths are
-// even (T even), so every copy is 16-byte aligned and sized.
+// Bulk copies of one tile's packed rows: this CTA's 64 K rows and all 128 V
+// rows.  Every run of consecutive keys inside one frame is contiguous in the
+// planes; run starts and lengths are even (T even), so every copy is 16-byte
+// aligned and sized.
+__device__ __forceinline__ void copy_runs(const AttnLaunch &a, int b, size_t head_row0, int k0,
+                                          int k1, uint8_t *dst_c, uint8_t *dst_s,
+                                          const uint8_t *codes, const uint8_t *scales,
+                                          uint64_t *full)
+{
+    for (int k = k0; k < k1;) {
+        const int f = div_fast(k, a.T, a.inv_T), tok = k - f * a.T;
+        const int n = min(a.T - tok, k1 - k);
+        const size_t g = head_row0 + (size_t)a.vis[b][f].slot * a.T + tok;
+        const int t0 = k - k0;
+        ptx::bulk_g2s(dst_c + t0 * 64, codes + g * 64, (uint32_t)n * 64, full);
+        ptx::bulk_g2s(dst_s + t0 * 8, scales + g * 8, (uint32_t)n * 8, full);
+        k += n;
+    }
+}
+
 __device__ void producer_role(Ctx &c)
 {
     const AttnLaunch &a = *c.a;
-    const uint8_t *kc = static_cast<const uint8_t *>(a.k_data);
-    const uint8_t *vc = static_cast<const uint8_t *>(a.v_data);
-    const uint8_t *ks = static_cast<const uint8_t *>(a.k_scales);
-    const uint8_t *vs = static_cast<const uint8_t *>(a.v_scales);
-    const size_t head_row0 = (size_t)(c.b * a.H + c.h) * a.R;
-    for (int j = 0; j < c.n_tiles; ++j) {
-        const int s = j % NSTAGE;
-        if (j >= NSTAGE && !wait(c, B_STG_EMPTY + s, ((j - NSTAGE) / NSTAGE) & 1)) return;
-        uint8_t *stg = c.smem + OFF_STG + s * STG_BYTES;
-        uint64_t *full = &c.ctl->bar[B_STG_FULL + s];
-        const int k0 = j * BN;
-        const int k1 = min(c.n_keys, k0 + BN);
-        ptx::mbar_arrive_expect_tx(full, (uint32_t)(k1 - k0) * 144u);
-        for (int k = k0; k < k1;) {
-            const int f = div_fast(k, a.T, a.inv_T), tok = k - f * a.T;
-            const int n = min(a.T - tok, k1 - k);
-            const size_t g = head_row0 + (size_t)a.vis[c.b][f].slot * a.T + tok;
-            const int t0 = k - k0;
-            ptx::bulk_g2s(stg + STG_KC + t0 * 64, kc + g * 64, (uint32_t)n * 64, full);
-            ptx::bulk_g2s(stg + STG_VC + t0 * 64, vc + g * 64, (uint32_t)n * 64, full);
-            ptx::bulk_g2s(stg + STG_KS + t0 * 8, ks + g * 8, (uint32_t)n * 8, full);
-            ptx::bulk_g2s(stg + STG_VS + t0 * 8, vs + g * 8, (uint32_t)n * 8, full);
-            k += n;
+    int g = 0;
+    for (int si = 0; si < c.ctl->n_seg; ++si) {
+        const Segment sg = c.ctl->seg[si];
+        const int n_keys = a.n_vis[sg.b] * a.T;
+        const size_t head_row0 = (size_t)(sg.b * a.H + sg.h) * a.R;
+        for (int tile = sg.t0; tile < sg.t1; ++tile, ++g) {
+            const int s = g % NSTAGE;
+            if (g >= NSTAGE && !wait(c, B_STG_EMPTY + s, ((g - NSTAGE) / NSTAGE) & 1)) return;
+            uint8_t *stg = c.smem + OFF_STG + s * STG_BYTES;
+            uint64_t *full = &c.ctl->bar[B_STG_FULL + s];
+            const int kk0 = min(n_keys, tile * BN + 64 * (int)c.rank);
+            const int kk1 = min(n_keys, tile * BN + 64 * (int)c.rank + 64);
+            const int vk0 = tile * BN;
+            const int vk1 = min(n_keys, vk0 + BN);
+            ptx::mbar_arrive_expect_tx(full, (uint32_t)((kk1 - kk0) + (vk1 - vk0)) * 72u);
+            copy_runs(a, sg.b, head_row0, kk0, kk1, stg + STG_KC, stg + STG_KS,
+                      static_cast<const uint8_t *>(a.k_data),
+                      static_cast<const uint8_t *>(a.k_scales), full);
+            copy_runs(a, sg.b, head_row0, vk0, vk1, stg + STG_VC, stg + STG_VS,
+                      static_cast<const uint8_t *>(a.v_data),
+                      static_cast<const uint8_t *>(a.v_scales), full);
         }
     }
 }
@@ -523,167 +652,278 @@ __device__ void producer_role(Ctx &c)
 __device__ void mma_role(Ctx &c)
 {
     const uint32_t tmem = c.ctl->tmem_base;
-    constexpr uint32_t idS = ptx::idesc_f16(kOperandF16, BM, BN, 0);
-    constexpr uint32_t idO = ptx::idesc_f16(kOperandF16, BM, 128, 1);
+    constexpr uint32_t idS = ptx::idesc_f16(kOperandF16, 2 * BM, BN, 0);
+    constexpr uint32_t idO = ptx::idesc_f16(kOperandF16, 2 * BM, 128, 1);
     const uint32_t ks = c.sbase + OFF_K;
     const uint32_t vs = c.sbase + OFF_V;
+    const uint16_t both = 0x3;
 
-    // S_tq = Q_tq K^T: A = Q from TMEM (8 x 16 channels), B = K tile, K-major
-    auto issue_s = [&](int tq, int kb) {
-        const uint32_t kt = ks + kb * KV_TILE;
+    // S_buf = Q K^T: A = Q (TMEM, 8 x 16 channels), B = the K halves, K-major
+    auto issue_s = [&](int buf, int kb) {
+        const uint32_t kt = ks + kb * K_TILE;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-            ptx::mma_f16_ts(tmem + TM_S + tq * 64, tmem + TM_Q + tq * 64 + kk * 8,
-                            ptx::smem_desc_sw128(kt + (kk >> 2) * KV_HALF + (kk & 3) * 32, 16,
-                                                 1024),
-                            idS, kk > 0);
-        ptx::mma_commit(&c.ctl->bar[B_S + tq]);
+            ptx::mma2_f16_ts(tmem + TM_S + buf * 128, tmem + TM_Q + kk * 8,
+                             ptx::smem_desc_sw128(kt + (kk >> 2) * K_HALF + (kk & 3) * 32, 16,
+                                                  1024),
+                             idS, kk > 0);
+        ptx::mma2_commit_mc(&c.ctl->bar[B_S + buf], both);
+        ptx::mma2_commit_mc(&c.ctl->bar[B_KFREE + kb], both);
     };
-    // O_tq += P_tq V: A = P from TMEM (4 x 16 keys), B = V tile, MN-major
-    auto issue_pv = [&](int tq, int vb, bool first) {
-        const uint32_t vt = vs + vb * KV_TILE;
+    // O += P V: A = P (TMEM over S_buf, 8 x 16 keys), B = the V halves, MN-major
+    auto issue_pv = [&](int buf, int vb, bool first) {
+        const uint32_t vt = vs + vb * V_TILE;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-            ptx::mma_f16_ts(tmem + TM_O + tq * 128, tmem + TM_S + tq * 64 + kk * 8,
-                            ptx::smem_desc_sw128(vt + kk * 2048, KV_HALF, 1024), idO,
-                            (!first || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk)
+            ptx::mma2_f16_ts(tmem + TM_O, tmem + TM_S + buf * 128 + kk * 8,
+                             ptx::smem_desc_sw128(vt + kk * 2048, V_TILE, 1024), idO,
+                             (!first || kk > 0) ? 1u : 0u);
+        ptx::mma2_commit_mc(&c.ctl->bar[B_VFREE + vb], both);
     };
 
-    bool ok = wait(c, B_Q, 0) && wait(c, B_KFULL, 0);
-    ptx::tc_fence_after();
-    if (ok) {
-        issue_s(0, 0);
-        issue_s(1, 0);
-        ptx::mma_commit(&c.ctl->bar[B_KFREE]);
-    }
-    for (int j = 0; ok && j < c.n_tiles; ++j) {
-        const int jn = j + 1, vb = j & 1;
-        if (!(ok = wait(c, B_VFULL + vb, (j >> 1) & 1) && wait(c, B_P, j & 1))) break;
+    int g = 0;
+    bool ok = true;
+    for (int si = 0; ok && si < c.ctl->n_seg; ++si) {
+        const Segment sg = c.ctl->seg[si];
+        const int n = sg.t1 - sg.t0, g0 = g;
+        if (!(ok = wait(c, B_QREADY, si & 1) && wait(c, B_KFULL + (g0 & 1), (g0 >> 1) & 1)))
+            break;
         ptx::tc_fence_after();
-        issue_pv(0, vb, j == 0);
-        if (jn < c.n_tiles) {
-            if (!(ok = wait(c, B_KFULL + (jn & 1), (jn >> 1) & 1))) break;
+        issue_s(g0 & 1, g0 & 1);
+        for (int i = 0; i < n; ++i, ++g) {
+            if (i + 1 < n) {
+                if (!(ok = wait(c, B_KFULL + ((g + 1) & 1), ((g + 1) >> 1) & 1))) break;
+                ptx::tc_fence_after();
+                issue_s((g + 1) & 1, (g + 1) & 1);
+            }
+            if (!(ok = wait(c, B_VFULL + (g & 1), (g >> 1) & 1) &&
+                       wait(c, B_P + (g & 1), (g >> 1) & 1) &&
+                       (i > 0 || si == 0 || wait(c, B_OFREE, (si - 1) & 1))))
+                break;
             ptx::tc_fence_after();
-            issue_s(0, jn & 1);
+            issue_pv(g & 1, g & 1, i == 0);
         }
-        if (!(ok = wait(c, B_P + 1, j & 1))) break;
-        ptx::tc_fence_after();
-        issue_pv(1, vb, j == 0);
-        ptx::mma_commit(&c.ctl->bar[B_VFREE + vb]);
-        if (jn < c.n_tiles) {
-            issue_s(1, jn & 1);
-            ptx::mma_commit(&c.ctl->bar[B_KFREE + (jn & 1)]);
-        }
+        if (!ok) break;
+        ptx::mma2_commit_mc(&c.ctl->bar[B_QFREE], both);
+        ptx::mma2_commit_mc(&c.ctl->bar[B_ODONE], both);
     }
-    if (ok) ptx::mma_commit(&c.ctl->bar[B_ODONE]);
-    // every MMA this thread issued has finished before TMEM is released
-    ptx::mma_commit(&c.ctl->bar[B_MMADONE]);
-    const int never = 0;
-    ptx::mbar_wait(&c.ctl->bar[B_MMADONE], 0, &never, WAIT_LIMIT_NS);
+    // every MMA issued has finished (in both CTAs) before TMEM is released
+    ptx::mma2_commit_mc(&c.ctl->bar[B_MMADONE], both);
 }
 
 // ------------------------------------------------------------ softmax
 
-template <bool FP4>
-__device__ void softmax_role(Ctx &c)
+__device__ __forceinline__ void rescale_o(uint32_t tO, float alpha)
 {
-    const AttnLaunch &a = *c.a;
-    const int warp = threadIdx.x >> 5;
-    const int tq = warp >> 2;                       // Q tile A (0) or B (1)
-    const int r = threadIdx.x & 127;
-    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tmem = c.ctl->tmem_base;
-    const uint32_t tS = tmem + TM_S + tq * 64 + lane_off;
-    const uint32_t tO = tmem + TM_O + tq * 128 + lane_off;
-    const int gi = c.b * a.H + c.h;
-    const float sgk = FP4 ? a.s_g[gi] : 1.0f;
-    const float sgv = FP4 ? a.s_g[a.B * a.H + gi] : 1.0f;
-    const float scale = sgk * 1.4426950408889634f * 0.08838834764831845f;   // log2(e)/sqrt(128)
-    float m = -INFINITY, l = 0.0f;
-    for (int j = 0; j < c.n_tiles; ++j) {
-        if (!wait_warp(c, B_S + tq, j & 1)) return;
-        ptx::tc_fence_after();
-        float s[64];
-        ptx::tmem_ld32(tS, reinterpret_cast<uint32_t *>(s));
-        ptx::tmem_ld32(tS + 32, reinterpret_cast<uint32_t *>(s) + 32);
-        ptx::tmem_wait_ld();
-        const int nv = c.n_keys - j * BN;
-        if (nv < BN) {
-#pragma unroll
-            for (int i = 0; i < 64; ++i)
-                if (i >= nv) s[i] = -INFINITY;
-        }
-        float mx = s[0];
-#pragma unroll
-        for (int i = 1; i < 64; ++i) mx = fmaxf(mx, s[i]);
-        const float mt = mx * scale;
-        if (__any_sync(0xFFFFFFFFu, mt > m + 8.0f)) {
-            const float mn = fmaxf(m, mt);
-            const float alpha = ex2(m - mn);     // 0 on the first tile
-            l *= alpha;
-            m = mn;
-            if (j > 0) {
-                // PV of the previous tile finished before this tile's S did
-#pragma unroll 1
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t o[32];
-                    ptx::tmem_ld32(tO + q * 32, o);
-                    ptx::tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    ptx::tmem_st32(tO + q * 32, o);
-                }
-            }
-        }
-        uint32_t pk[32];
-        float sum = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const float p0 = ex2(fmaf(s[2 * i], scale, -m));
-            const float p1 = ex2(fmaf(s[2 * i + 1], scale, -m));
-            sum += p0 + p1;
-            pk[i] = pack_f16(p0, p1);
-        }
-        l += sum;
-        ptx::tmem_st32(tS, pk);
-        ptx::tmem_wait_st();
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(&c.ctl->bar[B_P + tq]);
-    }
-    if (!wait_warp(c, B_ODONE, 0)) return;
-    ptx::tc_fence_after();
-    const int row = c.q0 + tq * BM + r;
-    const float fin = sgv / l;
-    uint4 *dst = reinterpret_cast<uint4 *>(a.out) + (((size_t)c.b * a.Lq + row) * a.H + c.h) * 16;
 #pragma unroll 1
     for (int q = 0; q < 4; ++q) {
         uint32_t o[32];
         ptx::tmem_ld32(tO + q * 32, o);
         ptx::tmem_wait_ld();
-        if (row < a.Lq) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                uint32_t w[4];
+        for (int i = 0; i < 32; i += 2) {
+            const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])),
+                                        make_float2(alpha, alpha));
+            o[i] = __float_as_uint(v.x);
+            o[i + 1] = __float_as_uint(v.y);
+        }
+        ptx::tmem_st32(tO + q * 32, o);
+    }
+}
+
+__device__ __forceinline__ void store_row_bf16(uint4 *dst, const float *acc, float fin)
+{
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float x = __uint_as_float(o[8 * i + 2 * k]) * fin;
-                    const float y = __uint_as_float(o[8 * i + 2 * k + 1]) * fin;
-                    __nv_bfloat162 bb = __floats2bfloat162_rn(x, y);
-                    w[k] = *reinterpret_cast<uint32_t *>(&bb);
+    for (int i = 0; i < 4; ++i) {
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            __nv_bfloat162 bb = __floats2bfloat162_rn(acc[8 * i + 2 * k] * fin,
+                                                      acc[8 * i + 2 * k + 1] * fin);
+            w[k] = *reinterpret_cast<uint32_t *>(&bb);
+        }
+        dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+template <bool FP4>
+__device__ void softmax_role(Ctx &c)
+{
+    const AttnLaunch &a = *c.a;
+    const int r = threadIdx.x;                      // 0..127 = TMEM lane
+    const uint32_t lane_off = (uint32_t)(r & ~31) << 16;
+    const uint32_t tmem = c.ctl->tmem_base + lane_off;
+    const uint32_t tO = tmem + TM_O;
+    float *ws = static_cast<float *>(a.workspace);
+    int *counters = reinterpret_cast<int *>(ws + (size_t)a.n_slots * 2 * 2 * BM * PART_FLOATS);
+    const long long target = (total_tiles(a) + a.n_slots - 1) / a.n_slots;
+    int g = 0;
+    for (int si = 0; si < c.ctl->n_seg; ++si) {
+        const Segment sg = c.ctl->seg[si];
+        const int n_keys = a.n_vis[sg.b] * a.T;
+        const int gi = sg.b * a.H + sg.h;
+        const float sgk = FP4 ? a.s_g[gi] : 1.0f;
+        const float sgv = FP4 ? a.s_g[a.B * a.H + gi] : 1.0f;
+        const float scale = sgk * 1.4426950408889634f * 0.08838834764831845f;   // log2(e)/sqrt(128)
+        float m = -INFINITY, l = 0.0f;
+        for (int tile = sg.t0; tile < sg.t1; ++tile, ++g) {
+            const int buf = g & 1;
+            if (!wait_warp(c, B_S + buf, (g >> 1) & 1)) return;
+            ptx::tc_fence_after();
+            const uint32_t tS = tmem + TM_S + buf * 128;
+            const int nv = n_keys - tile * BN;   // valid keys of this tile (may exceed 128)
+            // pass 1: row max over the valid logits
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                float s[32];
+                ptx::tmem_ld32(tS + q * 32, reinterpret_cast<uint32_t *>(s));
+                ptx::tmem_wait_ld();
+                if (nv < BN) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (q * 32 + i >= nv) s[i] = -INFINITY;
                 }
-                dst[q * 4 + i] = make_uint4(w[0], w[1], w[2], w[3]);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], s[i]);
+            }
+            const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale;
+            if (__any_sync(0xFFFFFFFFu, mt > m + 8.0f)) {
+                const float mn = fmaxf(m, mt);
+                const float alpha = ex2(m - mn);     // 0 on the first tile of a segment
+                l *= alpha;
+                m = mn;
+                if (tile > sg.t0) {
+                    // O holds the previous tile's PV once its V buffer was freed
+                    const int gp = g - 1;
+                    if (!wait_warp(c, B_VFREE + (gp & 1), (gp >> 1) & 1)) return;
+                    ptx::tc_fence_after();
+                    rescale_o(tO, alpha);
+                }
+            }
+            // pass 2: P = 2^(s * scale - m) as f16 pairs over S (keys 2i, 2i+1 ->
+            // column i); the chunk q of 32 logits becomes columns [16q, 16q + 16)
+            const float2 sc2 = make_float2(scale, scale), nm2 = make_float2(-m, -m);
+            float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                float s[32];
+                ptx::tmem_ld32(tS + q * 32, reinterpret_cast<uint32_t *>(s));
+                ptx::tmem_wait_ld();
+                if (nv < BN) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (q * 32 + i >= nv) s[i] = -INFINITY;
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float2 t2 = __ffma2_rn(make_float2(s[2 * i], s[2 * i + 1]), sc2, nm2);
+                    const float2 p = make_float2(ex2(t2.x), ex2(t2.y));
+                    acc[i & 1] = __fadd2_rn(acc[i & 1], p);
+                    pk[i] = pack_f16(p.x, p.y);
+                }
+                ptx::tmem_st16(tS + q * 16, pk);
+            }
+            const float2 at = __fadd2_rn(acc[0], acc[1]);
+            l += at.x + at.y;
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            ptx::mbar_arrive_remote(lead(c, B_P + buf));
+        }
+        // epilogue of the segment
+        if (!wait_warp(c, B_ODONE, si & 1)) return;
+        ptx::tc_fence_after();
+        const int row = (2 * sg.p + (int)c.rank) * BM + r;
+        if (sg.n_chunks == 1) {
+            const float fin = sgv / l;
+            uint4 *dst = reinterpret_cast<uint4 *>(a.out) +
+                         (((size_t)sg.b * a.Lq + (row < a.Lq ? row : 0)) * a.H + sg.h) * 16;
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                float o[32];
+                ptx::tmem_ld32(tO + q * 32, reinterpret_cast<uint32_t *>(o));
+                ptx::tmem_wait_ld();
+                if (row < a.Lq) store_row_bf16(dst + q * 4, o, fin);
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive_remote(lead(c, B_OFREE));
+            if (a.lse && row < a.Lq)
+                a.lse[(size_t)gi * a.Lq + row] = (m + __log2f(l)) * 0.6931471805599453f;
+        } else {
+            // partial record: unnormalised O, running max, sum
+            float *rec = ws + (((size_t)sg.part * 2 + c.rank) * BM + r) * PART_FLOATS;
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                uint32_t o[32];
+                ptx::tmem_ld32(tO + q * 32, o);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) __stcg(rec + q * 32 + i, __uint_as_float(o[i]));
+            }
+            __stcg(rec + 128, m);
+            __stcg(rec + 129, l);
+            ptx::tc_fence_before();
+            ptx::mbar_arrive_remote(lead(c, B_OFREE));
+            __threadfence();
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            int *ctr = counters + 2 * sg.first_slot + c.rank;
+            if (r == 0) c.ctl->merge_flag = (atomicAdd(ctr, 1) == sg.n_chunks - 1) ? 1 : 0;
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (c.ctl->merge_flag) {
+                __threadfence();
+                // merge every chunk's record for this row (this one included)
+                float mm = -INFINITY;
+                for (int k = 0; k < sg.n_chunks; ++k) {
+                    const float *rk =
+                        ws + (((size_t)chunk_part(sg, k, target) * 2 + c.rank) * BM + r) * PART_FLOATS;
+                    mm = fmaxf(mm, __ldcg(rk + 128));
+                }
+                float wk[8];
+                float lsum = 0.0f;
+                const int nk = sg.n_chunks;
+                for (int k = 0; k < nk && k < 8; ++k) {
+                    const float *rk =
+                        ws + (((size_t)chunk_part(sg, k, target) * 2 + c.rank) * BM + r) * PART_FLOATS;
+                    wk[k] = ex2(__ldcg(rk + 128) - mm);
+                    lsum += wk[k] * __ldcg(rk + 129);
+                }
+                for (int k = 8; k < nk; ++k) {
+                    const float *rk =
+                        ws + (((size_t)chunk_part(sg, k, target) * 2 + c.rank) * BM + r) * PART_FLOATS;
+                    lsum += ex2(__ldcg(rk + 128) - mm) * __ldcg(rk + 129);
+                }
+                const float fin = sgv / lsum;
+                uint4 *dst = reinterpret_cast<uint4 *>(a.out) +
+                             (((size_t)sg.b * a.Lq + (row < a.Lq ? row : 0)) * a.H + sg.h) * 16;
+#pragma unroll 1
+                for (int q = 0; q < 4; ++q) {
+                    float o[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = 0.0f;
+                    for (int k = 0; k < nk; ++k) {
+                        const float *rk =
+                            ws + (((size_t)chunk_part(sg, k, target) * 2 + c.rank) * BM + r) *
+                                     PART_FLOATS;
+                        const float w = k < 8 ? wk[k] : ex2(__ldcg(rk + 128) - mm);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] = fmaf(w, __ldcg(rk + q * 32 + i), o[i]);
+                    }
+                    if (row < a.Lq) store_row_bf16(dst + q * 4, o, fin);
+                }
+                if (a.lse && row < a.Lq)
+                    a.lse[(size_t)gi * a.Lq + row] = (mm + __log2f(lsum)) * 0.6931471805599453f;
+                if (r == 0) *ctr = 0;      // leave the workspace zeroed
             }
         }
     }
-    if (a.lse && row < a.Lq)
-        a.lse[(size_t)(c.b * a.H + c.h) * a.Lq + row] = (m + __log2f(l)) * 0.6931471805599453f;
 }
 
 // ------------------------------------------------------------ kernel
 
 template <bool FP4>
-__global__ void __launch_bounds__(NTHREADS, 1) k_chunk_attn(const __grid_constant__ AttnLaunch a)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+    k_chunk_attn(const __grid_constant__ AttnLaunch a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -692,69 +932,64 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chunk_attn(const __grid_constan
     c.a = &a;
     c.smem = smem;
     c.sbase = ptx::smem_u32(smem);
-    c.b = blockIdx.z;
-    c.h = blockIdx.y;
-    c.q0 = blockIdx.x * 2 * BM;
-    c.n_keys = a.n_vis[c.b] * a.T;
-    c.n_tiles = (c.n_keys + BN - 1) / BN;
+    c.rank = ptx::cluster_ctarank();
+    c.slot = blockIdx.x >> 1;
     c.tab_f = OFF_TAB;
     c.tab_h = c.tab_f + a.n_fpos * PAIRS_F * 8;
     c.tab_w = c.tab_h + a.grid_h * PAIRS_H * 8;
     const uint32_t ctl_off = (c.tab_w + a.grid_w * PAIRS_W * 8 + 63) & ~63u;
     c.ctl = reinterpret_cast<SharedCtl *>(smem + ctl_off);
+    c.lead_bar = ptx::mapa(ptx::smem_u32(&c.ctl->bar[0]), 0);
+    c.peer_abort = ptx::mapa(ptx::smem_u32(&c.ctl->abort), c.rank ^ 1u);
     const int warp = threadIdx.x >> 5;
 
     if (threadIdx.x == 0) {
-        // arrival counts: K converters (128) for Q and K full; V converters
-        // (64) for V full; both (192) for staging empty; the producer (1, plus
-        // bytes) for staging full; tcgen05.commit (1) for what the tensor core
-        // signals; a softmax group (128) for P.
-        ptx::mbar_init(&c.ctl->bar[B_Q], 128);
-        for (int s = 0; s < NSTAGE; ++s) {
-            ptx::mbar_init(&c.ctl->bar[B_STG_FULL + s], 1);
-            ptx::mbar_init(&c.ctl->bar[B_STG_EMPTY + s], 192);
+        // arrival counts: the even CTA's barriers that both CTAs feed take 256
+        // (128 threads of each); tcgen05.commit arrives once; staging full is
+        // the producer (1, plus bytes); staging empty the K and V converters.
+        for (int i = 0; i < N_BARS; ++i) {
+            uint32_t n = 1;
+            if (i < B_S) n = 256;
+            if (i >= B_STG_EMPTY) n = 256;
+            ptx::mbar_init(&c.ctl->bar[i], n);
         }
-        for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(&c.ctl->bar[B_KFULL + i], 128);
-            ptx::mbar_init(&c.ctl->bar[B_KFREE + i], 1);
-            ptx::mbar_init(&c.ctl->bar[B_VFULL + i], 64);
-            ptx::mbar_init(&c.ctl->bar[B_VFREE + i], 1);
-            ptx::mbar_init(&c.ctl->bar[B_S + i], 1);
-            ptx::mbar_init(&c.ctl->bar[B_P + i], 128);
-        }
-        ptx::mbar_init(&c.ctl->bar[B_ODONE], 1);
-        ptx::mbar_init(&c.ctl->bar[B_MMADONE], 1);
         c.ctl->abort = 0;
+        build_schedule(c);
         ptx::fence_mbar_init();
     }
     build_tables<FP4>(c);
-    if (warp == 15) {
-        ptx::tmem_alloc(&c.ctl->tmem_base, 512);
-        ptx::tmem_relinquish();
+    if (warp == 13) {
+        ptx::tmem_alloc2(&c.ctl->tmem_base, 512);
+        ptx::tmem_relinquish2();
     }
     ptx::tc_fence_before();
     __syncthreads();
+    ptx::cluster_sync();          // peer barriers initialised before any remote arrive
     ptx::tc_fence_after();
 
-    if (c.n_tiles > 0) {
-        if (warp < 8) {
-            softmax_role<FP4>(c);
-        } else if (warp < 12) {
-            k_converter_role<FP4>(c);
-        } else if (warp < 14) {
-            v_converter_role<FP4>(c);
-        } else if (warp == 14) {
-            if (FP4 && (threadIdx.x & 31) == 0) producer_role(c);
-        } else if ((threadIdx.x & 31) == 0) {
-            mma_role(c);
-        }
+    if (warp < 4) {
+        softmax_role<FP4>(c);
+    } else if (warp < 8) {
+        k_converter_role<FP4>(c);
+    } else if (warp < 12) {
+        v_converter_role<FP4>(c);
+    } else if (warp == 12) {
+        if (FP4 && (threadIdx.x & 31) == 0) producer_role(c);
+    } else if (warp == 13) {
+        if (c.rank == 0 && (threadIdx.x & 31) == 0) mma_role(c);
+        __syncwarp();
+        // both CTAs: every MMA touching this CTA's TMEM has completed
+        const int never = 0;
+        if ((threadIdx.x & 31) == 0)
+            ptx::mbar_wait_cluster(&c.ctl->bar[B_MMADONE], 0, &never, WAIT_LIMIT_NS);
+        __syncwarp();
     }
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == 15) {
-        __syncwarp();
+    ptx::cluster_sync();          // no CTA leaves while its peer may touch its memory
+    if (warp == 13) {
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(c.ctl->tmem_base, 512);
+        ptx::tmem_dealloc2(c.ctl->tmem_base, 512);
     }
 }
 
@@ -768,12 +1003,26 @@ cudaError_t launch(const AttnLaunch &a, cudaStream_t s)
     cudaError_t e = cudaFuncSetAttribute(k_chunk_attn<FP4>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
-    const dim3 grid((a.Lq + 2 * BM - 1) / (2 * BM), a.H, a.B);
+    const dim3 grid(2 * a.n_slots, 1, 1);
     k_chunk_attn<FP4><<<grid, NTHREADS, bytes, s>>>(a);
     return cudaGetLastError();
 }
 
 }  // namespace
+
+size_t attention_workspace_bytes(int n_slots)
+{
+    return (size_t)n_slots * 2 * 2 * BM * PART_FLOATS * sizeof(float) +
+           (size_t)n_slots * 2 * sizeof(int);
+}
+
+int attention_slots(int device)
+{
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
+        return 0;
+    return sms / 2;
+}
 
 cudaError_t launch_chunk_attention(const AttnLaunch &a, cudaStream_t s)
 {

@@ -15,7 +15,10 @@
 //   * multi-shot: a chunk of shot s sees the global sink, every frame of shot
 //     s and the last frame of each earlier shot; the first chunk of a shot
 //     s > 0 is pinned while that shot runs.
+#include <algorithm>
+#include <climits>
 #include <cmath>
+#include <cstdint>
 #include <cstring>
 
 #include "nvkv_internal.h"
@@ -145,12 +148,27 @@ nvkv_status append_common(const nvkv_desc *desc, const nvkv_cache *cache, nvkv_r
     return NVKV_OK;
 }
 
+// Persistent schedule of the attention kernel: CTA pairs (slots) and the
+// tiles per slot.  Each slot holds at most kMaxSegments work segments, so
+// very small items raise the slot count (extra pairs run as later waves).
+constexpr int kTileKeys = 128;
+constexpr int kMaxSegments = 94;     // the kernel holds 96; two spare
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+int schedule_slots(int dev_slots, int64_t total_tiles, int64_t min_item_tiles)
+{
+    int64_t n = dev_slots;
+    if (min_item_tiles > 0) n = std::max<int64_t>(n, ceil_div(total_tiles, kMaxSegments * min_item_tiles));
+    return (int)std::min<int64_t>(n, 1 << 20);
+}
+
+int query_pairs(const nvkv_desc *d) { return (int)ceil_div(ceil_div((int64_t)d->C * d->grid_h * d->grid_w, 128), 2); }
+
 nvkv_status attention_common(const nvkv_desc *desc, const nvkv_cache *cache,
                              const nvkv_ring *ring, const void *q, void *out, float *lse,
                              void *ws, size_t ws_bytes, cudaStream_t stream, int dtype)
 {
-    (void)ws;
-    (void)ws_bytes;
     nvkv_status st = check_desc(desc);
     if (st != NVKV_OK) return st;
     if (desc->kv_dtype != dtype) return NVKV_ERR_STATE;
@@ -215,6 +233,21 @@ nvkv_status attention_common(const nvkv_desc *desc, const nvkv_cache *cache,
         a.q_pos0[b] = s.n_resident - desc->C;
         if (s.n_resident > a.n_fpos) a.n_fpos = s.n_resident;
     }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVKV_ERR_CUDA;
+    const int dev_slots = nvkv::attention_slots(dev);
+    if (dev_slots < 1) return NVKV_ERR_CUDA;
+    a.n_pairs = query_pairs(desc);
+    int64_t total = 0, min_tiles = INT64_MAX;
+    for (int b = 0; b < desc->B; ++b) {
+        const int64_t nkt = ceil_div((int64_t)a.n_vis[b] * a.T, kTileKeys);
+        total += (int64_t)desc->H * a.n_pairs * nkt;
+        min_tiles = std::min(min_tiles, nkt);
+    }
+    a.n_slots = schedule_slots(dev_slots, total, min_tiles);
+    if (!ws || ws_bytes < nvkv::attention_workspace_bytes(a.n_slots)) return NVKV_ERR_CAPACITY;
+    if (reinterpret_cast<uintptr_t>(ws) & 15u) return NVKV_ERR_ALIGNMENT;
+    a.workspace = ws;
     if (nvkv::launch_chunk_attention(a, stream) != cudaSuccess) return NVKV_ERR_CUDA;
     return NVKV_OK;
 }
@@ -373,8 +406,18 @@ nvkv_status bf16_kv_append(const nvkv_desc *desc, const nvkv_cache *cache, nvkv_
 
 size_t nvkv_attention_workspace_bytes(const nvkv_desc *desc)
 {
-    (void)desc;
-    return 0;
+    if (check_desc(desc) != NVKV_OK) return 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    const int dev_slots = nvkv::attention_slots(dev);
+    if (dev_slots < 1) return 0;
+    // bound over every ring state: at most S + W visible frames, at least the
+    // chunk's own C frames
+    const int64_t T = (int64_t)desc->grid_h * desc->grid_w;
+    const int64_t max_tiles = ceil_div((desc->S + desc->W) * T, kTileKeys);
+    const int64_t min_tiles = ceil_div(desc->C * T, kTileKeys);
+    const int64_t total = (int64_t)desc->B * desc->H * query_pairs(desc) * max_tiles;
+    return nvkv::attention_workspace_bytes(schedule_slots(dev_slots, total, min_tiles));
 }
 
 nvkv_status chunk_attention_nvfp4kv(const nvkv_desc *desc, const nvkv_cache *cache,

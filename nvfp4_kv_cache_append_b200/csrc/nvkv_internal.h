@@ -50,7 +50,15 @@ struct AttnLaunch {
     float inv_T, inv_grid_w;         // 1/T and 1/grid_w (division by reciprocal + fix-up)
     int n_fpos;                      // frame positions used: 0 .. n_fpos-1
     float theta[64];                 // RoPE angle per unit position of each channel pair
+    void *workspace;                 // split-item partials + counters (zero on first use)
+    int n_slots;                     // CTA pairs of the persistent schedule
+    int n_pairs;                     // 256-row query tile pairs per (b, h)
 };
+
+// Workspace of the chunk attention for a schedule of n_slots CTA pairs:
+// per slot two partial records of 2 x 128 rows x (128 + 2) f32, then counters.
+size_t attention_workspace_bytes(int n_slots);
+int attention_slots(int device);     // CTA pairs that can be resident at once
 
 cudaError_t launch_chunk_attention(const AttnLaunch &a, cudaStream_t s);
 
