@@ -30,7 +30,9 @@
 //                and scale rows into a 4-stage staging ring (NVFP4 only).
 //   warp 13      TMEM allocation (both CTAs) and, in the even CTA, the MMA
 //                issuer: S = Q K^T into one of two S buffers while the softmax
-//                reads the other, then O += P V.
+//                reads the other, then O += P V.  In the odd CTA its lane 0
+//                relays the P and O-free events to the even CTA.
+//   warps 14-15  odd CTA only: lane 0 relays the Q/K and the V events.
 // TMEM per CTA: Q (64 cols, f16 pairs) | S0 (128) | S1 (128) | O (128).
 // Dequantized values are exact in f16 (E2M1 code x E4M3 scale); the global
 // scales fold into the softmax scale (K) and the epilogue (V).
@@ -242,6 +244,14 @@ __device__ __forceinline__ bool wait(Ctx &c, int bar, uint32_t parity)
     set_abort(c);
     return false;
 }
+
+// Cross-CTA events (Q ready, K/V halves converted, P written, O read) are
+// counted on the even CTA's barrier.  Every thread arrives on its own CTA's
+// copy with a CTA-scope release (a few cycles); in the odd CTA one relay
+// thread per event stream waits for the local phase and forwards it with a
+// single cluster-scope release arrive (a few hundred cycles, paid once per
+// event instead of once per thread).
+__device__ __forceinline__ void arrive_x(Ctx &c, int bar) { ptx::mbar_arrive(&c.ctl->bar[bar]); }
 
 // wait by every lane of a warp, outcome made warp-uniform (the tcgen05 loads
 // and stores that follow are warp-collective)
@@ -546,7 +556,7 @@ __device__ void k_converter_role(Ctx &c)
         load_q_tmem<FP4>(c, sg.b, sg.h, (2 * sg.p + (int)c.rank) * BM + t, tmem + lane_off + TM_Q);
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
-        ptx::mbar_arrive_remote(lead(c, B_QREADY));
+        arrive_x(c, B_QREADY);
         for (int tile = sg.t0; tile < sg.t1; ++tile, ++g) {
             const int s = g % NSTAGE, kb = g & 1;
             const uint32_t stg = c.sbase + OFF_STG + s * STG_BYTES;
@@ -562,7 +572,7 @@ __device__ void k_converter_role(Ctx &c)
                 else conv_k_bf16<1>(c, sr, k, kdst);
             }
             ptx::fence_proxy_async_smem();
-            ptx::mbar_arrive_remote(lead(c, B_KFULL + kb));
+            arrive_x(c, B_KFULL + kb);
             if (FP4) ptx::mbar_arrive(&c.ctl->bar[B_STG_EMPTY + s]);
         }
     }
@@ -591,9 +601,52 @@ __device__ void v_converter_role(Ctx &c)
                 conv_v_bf16(c, k, (int)c.rank, kp, vdst);
             }
             ptx::fence_proxy_async_smem();
-            ptx::mbar_arrive_remote(lead(c, B_VFULL + vb));
+            arrive_x(c, B_VFULL + vb);
             if (FP4) ptx::mbar_arrive(&c.ctl->bar[B_STG_EMPTY + s]);
         }
+    }
+}
+
+// ------------------------------------------------------------ relays (odd CTA)
+
+__device__ __forceinline__ bool relay(Ctx &c, int bar, uint32_t parity)
+{
+    if (!wait(c, bar, parity)) return false;
+    ptx::mbar_arrive_remote(lead(c, bar));
+    return true;
+}
+
+// Q and K halves, in the order the K converters produce them
+__device__ void relay_qk_role(Ctx &c)
+{
+    int g = 0;
+    for (int si = 0; si < c.ctl->n_seg; ++si) {
+        const Segment sg = c.ctl->seg[si];
+        if (!relay(c, B_QREADY, si & 1)) return;
+        for (int tile = sg.t0; tile < sg.t1; ++tile, ++g)
+            if (!relay(c, B_KFULL + (g & 1), (g >> 1) & 1)) return;
+    }
+}
+
+__device__ void relay_v_role(Ctx &c)
+{
+    int g = 0;
+    for (int si = 0; si < c.ctl->n_seg; ++si) {
+        const Segment sg = c.ctl->seg[si];
+        for (int tile = sg.t0; tile < sg.t1; ++tile, ++g)
+            if (!relay(c, B_VFULL + (g & 1), (g >> 1) & 1)) return;
+    }
+}
+
+// P of every tile, then O released at the end of each segment
+__device__ void relay_p_role(Ctx &c)
+{
+    int g = 0;
+    for (int si = 0; si < c.ctl->n_seg; ++si) {
+        const Segment sg = c.ctl->seg[si];
+        for (int tile = sg.t0; tile < sg.t1; ++tile, ++g)
+            if (!relay(c, B_P + (g & 1), (g >> 1) & 1)) return;
+        if (!relay(c, B_OFREE, si & 1)) return;
     }
 }
 
@@ -829,7 +882,7 @@ __device__ void softmax_role(Ctx &c)
             l += at.x + at.y;
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
-            ptx::mbar_arrive_remote(lead(c, B_P + buf));
+            arrive_x(c, B_P + buf);
         }
         // epilogue of the segment
         if (!wait_warp(c, B_ODONE, si & 1)) return;
@@ -847,7 +900,7 @@ __device__ void softmax_role(Ctx &c)
                 if (row < a.Lq) store_row_bf16(dst + q * 4, o, fin);
             }
             ptx::tc_fence_before();
-            ptx::mbar_arrive_remote(lead(c, B_OFREE));
+            arrive_x(c, B_OFREE);
             if (a.lse && row < a.Lq)
                 a.lse[(size_t)gi * a.Lq + row] = (m + __log2f(l)) * 0.6931471805599453f;
         } else {
@@ -864,7 +917,7 @@ __device__ void softmax_role(Ctx &c)
             __stcg(rec + 128, m);
             __stcg(rec + 129, l);
             ptx::tc_fence_before();
-            ptx::mbar_arrive_remote(lead(c, B_OFREE));
+            arrive_x(c, B_OFREE);
             __threadfence();
             asm volatile("bar.sync 1, 128;" ::: "memory");
             int *ctr = counters + 2 * sg.first_slot + c.rank;
@@ -944,12 +997,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     const int warp = threadIdx.x >> 5;
 
     if (threadIdx.x == 0) {
-        // arrival counts: the even CTA's barriers that both CTAs feed take 256
-        // (128 threads of each); tcgen05.commit arrives once; staging full is
-        // the producer (1, plus bytes); staging empty the K and V converters.
+        // arrival counts: a cross-CTA event takes the 128 threads of its role
+        // in this CTA, plus, in the even CTA, the odd CTA's relay;
+        // tcgen05.commit arrives once; staging full is the producer (1, plus
+        // bytes); staging empty the K and V converters.
         for (int i = 0; i < N_BARS; ++i) {
             uint32_t n = 1;
-            if (i < B_S) n = 256;
+            if (i < B_S) n = c.rank == 0 ? 129 : 128;
             if (i >= B_STG_EMPTY) n = 256;
             ptx::mbar_init(&c.ctl->bar[i], n);
         }
@@ -976,13 +1030,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     } else if (warp == 12) {
         if (FP4 && (threadIdx.x & 31) == 0) producer_role(c);
     } else if (warp == 13) {
-        if (c.rank == 0 && (threadIdx.x & 31) == 0) mma_role(c);
+        if ((threadIdx.x & 31) == 0) {
+            if (c.rank == 0) mma_role(c);
+            else relay_p_role(c);
+        }
         __syncwarp();
         // both CTAs: every MMA touching this CTA's TMEM has completed
         const int never = 0;
         if ((threadIdx.x & 31) == 0)
             ptx::mbar_wait_cluster(&c.ctl->bar[B_MMADONE], 0, &never, WAIT_LIMIT_NS);
         __syncwarp();
+    } else if (c.rank == 1 && (threadIdx.x & 31) == 0) {
+        if (warp == 14) relay_qk_role(c);
+        else relay_v_role(c);
     }
     ptx::tc_fence_before();
     __syncthreads();
