@@ -11,10 +11,21 @@
 // stored as code 0.  The FP32 operations are IEEE round-to-nearest (no
 // contraction, true division), so the codes are bit-exact.
 //
-// Memory: HBM-bound.  Each thread owns one 16-element block: two 16-byte
-// loads of bf16 input (a warp reads 1 KB contiguous), one 8-byte code store
-// and one scale byte (eight threads of a token-head write 64 contiguous code
-// bytes).  Rows go straight into the physical frame slot (no staging).
+// Memory: HBM-bound.  Each thread owns two adjacent 16-element blocks: four
+// 16-byte loads of bf16 input (a warp reads 2 KB contiguous), one 16-byte
+// code store and one 2-byte scale store (four threads of a token-head write
+// its 64 contiguous code bytes).  Rows go straight into the physical frame
+// slot (no staging).
+//
+// The 16 quotients x_i / (s_b s_g) of a block share their divisor, so they
+// are taken by Markstein's correctly rounded division (P. Markstein, "IA-64
+// and Elementary Functions", 2000: with r = RN(1/d) and q = RN(x r), the
+// residual e = x - q d is exact under an FMA and RN(q + e r) = RN(x / d)):
+// one reciprocal per block, three FMA-pipe operations per element.  The
+// theorem needs the residual representable, which holds for 2^-64 <= d <=
+// 2^64 and quotients below 2^64 whenever |x / d| >= 1/16; below 1/16 every
+// candidate quotient encodes to code 0.  Blocks outside that range (tiny or
+// huge scales, infinities, NaN) take IEEE division.
 #include <cuda_bf16.h>
 
 #include "nvkv_internal.h"
@@ -101,6 +112,15 @@ __device__ __forceinline__ void unpack_bf16x8(uint4 a, float *x)
     }
 }
 
+// l / T for 0 <= l < 2^24 by a float reciprocal with a one-step fix-up
+__device__ __forceinline__ int frame_of(int l, const AppendLaunch &a)
+{
+    int f = __float2int_rz((float)l * a.inv_T);
+    if (f * a.T > l) --f;
+    else if ((f + 1) * a.T <= l) ++f;
+    return f;
+}
+
 // amax of the first chunk per (K/V, batch, head).  blockDim = (8H, ty),
 // grid = (gx, 2B).  amax must be zero on entry; float bits of non-negative
 // values order like unsigned integers, so atomicMax on the bits is exact.
@@ -130,50 +150,76 @@ __global__ void k_first_chunk_amax(const uint4 *__restrict__ k, const uint4 *__r
     if (tid < H && s_max[tid]) atomicMax(&amax[(t * B + b) * H + tid], s_max[tid]);
 }
 
-// blockDim = (8H, ty): threadIdx.x = h * 8 + block, threadIdx.y = token in the
-// CTA's token group.  grid = (ceil(Lq / ty), 2B): blockIdx.y = t * B + b with
-// t = 0 for K and 1 for V.
+// Codes of one 16-element block (bf16 in w0, w1) with global scale sg:
+// returns the E4M3 scale code, writes the 16 codes (element i in nibble i of
+// c.x | c.y << 32).
+__device__ __forceinline__ uint32_t quantize_block(uint4 w0, uint4 w1, float sg, uint2 &c)
+{
+    const float amax16 = halves_max(__vmaxu2(absmax_bits(w0), absmax_bits(w1)));
+    const float ratio = __fdiv_rn(amax16, __fmul_rn(6.0f, sg));
+    const uint32_t sb_code = e4m3_code(ratio);
+    const float sb = e4m3_value(sb_code);
+    c = make_uint2(0u, 0u);
+    if (sb == 0.0f) return sb_code;
+    const float d = __fmul_rn(sb, sg);
+    float x[16], y[16];
+    unpack_bf16x8(w0, x);
+    unpack_bf16x8(w1, x + 8);
+    const float r = __frcp_rn(d);
+    if (d >= 0x1p-64f && d <= 0x1p64f && amax16 * r < 0x1p64f) {
+        // y = RN(q + (x - q d) r) with q = RN(x r), two elements per operation
+        const float2 r2 = make_float2(r, r), nd2 = make_float2(-d, -d);
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+            const float2 xx = make_float2(x[i], x[i + 1]);
+            const float2 q = __fmul2_rn(xx, r2);
+            const float2 yy = __ffma2_rn(__ffma2_rn(q, nd2, xx), r2, q);
+            y[i] = yy.x;
+            y[i + 1] = yy.y;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) y[i] = __fdiv_rn(x[i], d);
+    }
+    c.x = drop_negative_zero(e2m1x8(y));
+    c.y = drop_negative_zero(e2m1x8(y + 8));
+    return sb_code;
+}
+
+// blockDim = (4H, ty): threadIdx.x = h * 4 + pair (blocks 2 pair, 2 pair + 1
+// of the token-head: 64 bytes in, 16 code bytes and 2 scale bytes out),
+// threadIdx.y = token in the CTA's token group.  grid = (ceil(Lq / ty), 2B):
+// blockIdx.y = t * B + b with t = 0 for K and 1 for V.
 __global__ void __launch_bounds__(512) k_nvfp4_append(const __grid_constant__ AppendLaunch a)
 {
     const int t = blockIdx.y / a.B, b = blockIdx.y - t * a.B;
     const int l = blockIdx.x * blockDim.y + threadIdx.y;
     if (l >= a.Lq) return;
-    const int h = threadIdx.x >> 3, blk = threadIdx.x & 7;
+    const int h = threadIdx.x >> 2, pr = threadIdx.x & 3;
     const uint4 *src = reinterpret_cast<const uint4 *>(t ? a.v : a.k) +
-                       (((size_t)b * a.Lq + l) * a.H + h) * 16 + blk * 2;
+                       (((size_t)b * a.Lq + l) * a.H + h) * 16 + pr * 4;
     const uint4 w0 = ld_stream(src), w1 = ld_stream(src + 1);
+    const uint4 w2 = ld_stream(src + 2), w3 = ld_stream(src + 3);
 
     const int gi = (t * a.B + b) * a.H + h;
     float sg;
     if (a.first) {
         sg = global_scale_from_amax(a.amax[gi]);
-        if (l == 0 && blk == 0) a.s_g[gi] = sg;
+        if (l == 0 && pr == 0) a.s_g[gi] = sg;
     } else {
         sg = a.s_g[gi];
     }
+    uint2 c0, c1;
+    const uint32_t s0 = quantize_block(w0, w1, sg, c0);
+    const uint32_t s1 = quantize_block(w2, w3, sg, c1);
 
-    const float amax16 = halves_max(__vmaxu2(absmax_bits(w0), absmax_bits(w1)));
-    const float ratio = __fdiv_rn(amax16, __fmul_rn(6.0f, sg));
-    const uint32_t sb_code = e4m3_code(ratio);
-    const float sb = e4m3_value(sb_code);
-    uint2 codes = make_uint2(0u, 0u);
-    if (sb != 0.0f) {
-        const float d = __fmul_rn(sb, sg);
-        float x[16], y[16];
-        unpack_bf16x8(w0, x);
-        unpack_bf16x8(w1, x + 8);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) y[i] = __fdiv_rn(x[i], d);
-        codes.x = drop_negative_zero(e2m1x8(y));
-        codes.y = drop_negative_zero(e2m1x8(y + 8));
-    }
-
-    const int frame = l / a.T, tok = l - frame * a.T;
+    const int frame = frame_of(l, a), tok = l - frame * a.T;
     const int slot = a.slot[b * a.C + frame];
     const size_t row = (size_t)(b * a.H + h) * a.R + (size_t)slot * a.T + tok;
-    uint8_t *cdst = static_cast<uint8_t *>(t ? a.v_data : a.k_data) + row * 64 + blk * 8;
-    *reinterpret_cast<uint2 *>(cdst) = codes;
-    static_cast<uint8_t *>(t ? a.v_scales : a.k_scales)[row * 8 + blk] = (uint8_t)sb_code;
+    *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(t ? a.v_data : a.k_data) + row * 64 + pr * 16) =
+        make_uint4(c0.x, c0.y, c1.x, c1.y);
+    *reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(t ? a.v_scales : a.k_scales) + row * 8 +
+                                  pr * 2) = (uint16_t)(s0 | (s1 << 8));
 }
 
 // bf16 twin: blockDim = (16H, ty), one 16-byte chunk per thread.
@@ -185,7 +231,7 @@ __global__ void __launch_bounds__(1024) k_bf16_append(const __grid_constant__ Ap
     const int h = threadIdx.x >> 4, c = threadIdx.x & 15;
     const uint4 *src = reinterpret_cast<const uint4 *>(t ? a.v : a.k) +
                        (((size_t)b * a.Lq + l) * a.H + h) * 16 + c;
-    const int frame = l / a.T, tok = l - frame * a.T;
+    const int frame = frame_of(l, a), tok = l - frame * a.T;
     const int slot = a.slot[b * a.C + frame];
     const size_t row = (size_t)(b * a.H + h) * a.R + (size_t)slot * a.T + tok;
     reinterpret_cast<uint4 *>(t ? a.v_data : a.k_data)[row * 16 + c] = ld_stream(src);
@@ -220,15 +266,19 @@ dim3 append_block(int H, int per_head)
 
 }  // namespace
 
-cudaError_t launch_nvfp4_append(const AppendLaunch &a, cudaStream_t s)
+cudaError_t launch_nvfp4_append(const AppendLaunch &a_in, cudaStream_t s)
 {
-    const dim3 blk = append_block(a.H, 8);
+    AppendLaunch a = a_in;
+    a.inv_T = 1.0f / (float)a.T;
+    const dim3 blk = append_block(a.H, 4);
     const dim3 grid((a.Lq + blk.y - 1) / blk.y, 2 * a.B);
     if (a.first) {
         cudaError_t e = cudaMemsetAsync(a.amax, 0, sizeof(uint32_t) * 2 * a.B * a.H, s);
         if (e != cudaSuccess) return e;
-        const dim3 g2(grid.x < 148 ? grid.x : 148, 2 * a.B);
-        k_first_chunk_amax<<<g2, blk, 0, s>>>(static_cast<const uint4 *>(a.k),
+        const dim3 blk8 = append_block(a.H, 8);
+        const unsigned gx = (a.Lq + blk8.y - 1) / blk8.y;
+        const dim3 g2(gx < 148 ? gx : 148, 2 * a.B);
+        k_first_chunk_amax<<<g2, blk8, 0, s>>>(static_cast<const uint4 *>(a.k),
                                               static_cast<const uint4 *>(a.v), a.amax, a.B, a.H,
                                               a.Lq);
     }
@@ -236,8 +286,10 @@ cudaError_t launch_nvfp4_append(const AppendLaunch &a, cudaStream_t s)
     return cudaGetLastError();
 }
 
-cudaError_t launch_bf16_append(const AppendLaunch &a, cudaStream_t s)
+cudaError_t launch_bf16_append(const AppendLaunch &a_in, cudaStream_t s)
 {
+    AppendLaunch a = a_in;
+    a.inv_T = 1.0f / (float)a.T;
     const dim3 blk = append_block(a.H, 16);
     const dim3 grid((a.Lq + blk.y - 1) / blk.y, 2 * a.B);
     k_bf16_append<<<grid, blk, 0, s>>>(a);

@@ -17,6 +17,7 @@ struct AppendLaunch {
     uint32_t *amax;                  // [2][B][H]
     float *s_g;                      // [2][B][H]
     int B, H, T, Lq, R, C;
+    float inv_T;                     // 1/T, set by the launchers (frame index by reciprocal)
     int first;                       // 1: measure amax and fix s_g
     int32_t slot[NVKV_MAX_BATCH * NVKV_MAX_CHUNK];  // [b * C + c] -> physical slot
 };

@@ -115,3 +115,32 @@ def test_bf16_twin_append_copies_exactly():
                 want = x[w][0, c * wl.T:(c + 1) * wl.T].transpose(0, 1)
                 got = lib.cache.codes(w)[0, :, rows].cpu()
                 assert torch.equal(got.view(torch.int16), want.contiguous().view(torch.int16))
+
+
+@pytest.mark.parametrize("first_scale,later_scale", [
+    (2.0 ** -100, 2.0 ** -100),   # tiny global scale: divisor below 2^-64 (IEEE-division blocks)
+    (2.0 ** -60, 1.0),            # later chunks far above the first: saturated codes
+    (1.0, 2.0 ** 40),             # block scales clamped at 448, quotients up to ~2^40
+    (1.0, 2.0 ** 70),             # quotients beyond 2^64 (IEEE-division blocks)
+    (2.0 ** 60, 2.0 ** 60),       # divisors near 2^64
+])
+def test_append_extreme_scales_bit_exact(first_scale, later_scale):
+    """Codes and scales stay bit-exact when the scales leave the usual range:
+    both the shared-reciprocal division and the IEEE-division fallback of the
+    append kernel meet the oracle's fl32(x / (s_b s_g))."""
+    import nvfp4_kv_cache_append_b200 as nv
+    wl = kvsynth.WORKLOADS["tiny"]
+    lib = LibStream(wl, nv.NVKV_KV_NVFP4)
+    ora = OracleStream(wl, seed=0, keep_inputs=False)
+    for step in range(1, 5):
+        x = kvsynth.chunk_qkv(wl, step, 0)
+        sc = first_scale if step == 1 else later_scale
+        k = (x["k"].float() * sc).to(torch.bfloat16)
+        v = (x["v"].float() * sc).to(torch.bfloat16)
+        new = ora.step(k=k, v=v, q=x["q"])
+        lib.cache.append(k.cuda(), v.cuda())
+        torch.cuda.synchronize()
+        if step == 1:
+            assert np.array_equal(lib.cache.global_scales().cpu().numpy(), ora.s_g)
+        _check_new_frames(lib, ora, new)
+    assert lib.cache.device_status() == 0
