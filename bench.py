@@ -128,6 +128,16 @@ def _dist_env():
     return ws, rank, local
 
 
+def bench_config(wl, kv, ws):
+    """The workload a line is measured on (shared by both arms)."""
+    n_keys = (wl.S + wl.W) * wl.T
+    return {"workload": f"{wl.name}: B{wl.B} H{wl.H} D128 T{wl.T} ({wl.grid_h}x{wl.grid_w}) "
+                        f"C{wl.C} S{wl.S} W{wl.W}, {wl.Lq} query tokens, {n_keys} keys",
+            "kv_cache": kv, "layers_cycled": N_LAYERS,
+            "l2": "inputs and caches larger than L2 (4 independent layers cycled)",
+            "parallelism": f"replicas x{ws}"}
+
+
 # --------------------------------------------------------------- our arm
 
 def run_ours(args):
@@ -274,11 +284,7 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "e2m1/e4m3 cache, f16 MMA, f32 accumulate" if fp4 else "bf16 MMA, f32 accumulate",
         "data": "synthetic (seeded bf16 N(0,1), 1% K outlier channels x8)",
-        "config": {"workload": f"{wl.name}: B{wl.B} H{wl.H} D128 T{wl.T} ({wl.grid_h}x{wl.grid_w}) "
-                               f"C{wl.C} S{wl.S} W{wl.W}, {wl.Lq} query tokens, {num['n_keys']} keys",
-                   "kv_cache": args.kv, "layers_cycled": N_LAYERS,
-                   "l2": "inputs and caches larger than L2 (4 independent layers cycled)",
-                   "parallelism": f"replicas x{ws}"},
+        "config": bench_config(wl, args.kv, ws),
         "attn_tflops": attn_tflops,
         "attn_ms": att_avg,
         "append_gbs": append_gbs,
@@ -305,56 +311,77 @@ def run_ours(args):
 
 # ------------------------------------------------------------ oracle arm
 
-def _oracle_sample(wl, n_rows, seed=0):
-    """Time the oracle on a bounded sample of one steady-state step."""
-    import numpy as np
+class OracleSample:
+    """Inputs of one steady-state step for timing the CPU oracle, drawn once
+    (outside every timed region); `run` times the oracle on a bounded sample
+    of the step: the quantize of `n_tok` of the chunk's tokens (K and V, every
+    head) and the attention of `n_rows` query tokens (every head) over all
+    the step's keys.  Returns query tok/s = 1 / (quantize s per token +
+    attention s per query token)."""
 
-    import kvsynth
-    import oracle
+    def __init__(self, wl, seed=0):
+        import numpy as np
 
-    x = kvsynth.chunk_qkv(wl, 1, seed)
-    kf, vf = x["k"].float().numpy(), x["v"].float().numpy()
-    t0 = time.perf_counter()
-    # quantize-append of the whole chunk (K and V, every head)
-    for arr in (kf, vf):
+        import kvsynth
+        self.wl = wl
+        x = kvsynth.chunk_qkv(wl, 1, seed)
+        self.kf = np.ascontiguousarray(x["k"].float().numpy()[0].transpose(1, 0, 2))   # [H][Lq][D]
+        self.vf = np.ascontiguousarray(x["v"].float().numpy()[0].transpose(1, 0, 2))
+        self.q = np.ascontiguousarray(x["q"].float().numpy()[0].transpose(1, 0, 2))
+        n_keys = (wl.S + wl.W) * wl.T
+        rng = np.random.default_rng(seed)
+        self.k = rng.standard_normal((n_keys, 128))
+        self.v = rng.standard_normal((n_keys, 128))
+        self.fpos = np.repeat(np.arange(wl.S + wl.W, dtype=np.int32), wl.T)
+        self.tok = np.tile(np.arange(wl.T, dtype=np.int32), wl.S + wl.W)
+        l = np.arange(wl.Lq)
+        self.qpos = (wl.S + wl.W - wl.C + l // wl.T).astype(np.int32)
+        self.qtok = (l % wl.T).astype(np.int32)
+        self.rng = rng
+
+    def run(self, n_tok, n_rows):
+        import numpy as np
+
+        import oracle
+        wl = self.wl
+        t0 = time.perf_counter()
+        for arr in (self.kf, self.vf):
+            for h in range(wl.H):
+                rows = arr[h, :n_tok]
+                oracle.quantize_rows(rows, oracle.global_scale(oracle.amax(rows)))
+        t_app = time.perf_counter() - t0
+        rows = self.rng.choice(wl.Lq, n_rows, replace=False)
+        t0 = time.perf_counter()
         for h in range(wl.H):
-            rows = np.ascontiguousarray(arr[0, :, h])
-            oracle.quantize_rows(rows, oracle.global_scale(oracle.amax(rows)))
-    t_app = time.perf_counter() - t0
-    # attention of n_rows query tokens (all heads) over 32760 keys
-    n_keys = (wl.S + wl.W) * wl.T
-    rng = np.random.default_rng(seed)
-    k = rng.standard_normal((n_keys, 128))
-    v = rng.standard_normal((n_keys, 128))
-    fpos = np.repeat(np.arange(wl.S + wl.W, dtype=np.int32), wl.T)
-    tok = np.tile(np.arange(wl.T, dtype=np.int32), wl.S + wl.W)
-    q = x["q"][0]
-    l = np.arange(wl.Lq)
-    qpos = (wl.S + wl.W - wl.C + l // wl.T).astype(np.int32)
-    qtok = (l % wl.T).astype(np.int32)
-    rows = rng.choice(wl.Lq, n_rows, replace=False)
-    t0 = time.perf_counter()
-    for h in range(wl.H):
-        oracle.attention_rows(q[:, h], k, v, fpos, tok, qpos, qtok, rows, wl.grid_w)
-    t_att = time.perf_counter() - t0
-    per_tok = t_app / wl.Lq + t_att / n_rows
-    return 1.0 / per_tok, t_app, t_att
+            oracle.attention_rows(self.q[h], self.k, self.v, self.fpos, self.tok, self.qpos,
+                                  self.qtok, rows, wl.grid_w)
+        t_att = time.perf_counter() - t0
+        return 1.0 / (t_app / n_tok + t_att / n_rows), t_app, t_att
+
+
+def _oracle_cores():
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
 
 
 def cpu_baseline(wl, seconds=20.0):
     import oracle
     oracle.build()
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    sample = OracleSample(wl)
     n_rows = max(8, int(seconds * 6))
-    value, t_app, t_att = _oracle_sample(wl, n_rows)
-    return {"value": value, "unit": "query tok/s", "cores": cores, "kind": "oracle",
+    value, t_app, t_att = sample.run(wl.Lq, n_rows)
+    return {"value": value, "unit": "query tok/s", "cores": _oracle_cores(), "kind": "oracle",
             "sample": f"one {wl.name} step: full-chunk quantize ({wl.Lq} tokens x {wl.H} heads, "
                       f"K and V) + attention of {n_rows} query tokens x {wl.H} heads over "
-                      f"{(wl.S + wl.W) * wl.T} keys; tok/s = 1 / (append s/token + attention s/token)",
+                      f"{(wl.S + wl.W) * wl.T} keys; tok/s = 1 / (quantize s/token + attention "
+                      f"s/token)",
             "append_s": t_app, "attention_s": t_att}
 
 
 def run_reference(args):
+    """The reference arm: the CPU oracle as it stands, on this arm's workload,
+    metric and config.  Each step is a bounded sample of the step (quantize
+    of a slice of the chunk, attention of a few query rows), sized so that the
+    whole run stays within about two minutes."""
     import kvsynth
     ws, rank, _ = _dist_env()
     if rank != 0:
@@ -362,27 +389,32 @@ def run_reference(args):
     wl = kvsynth.WORKLOADS[args.workload]
     import oracle
     oracle.build()
-    n_rows = 8
+    sample = OracleSample(wl)
+    # about 1.5 s of oracle work per step at 8 rows and the full chunk (8
+    # host cores); shrink the sample when many steps are asked for
+    budget_s = 120.0
+    frac = min(1.0, budget_s / (1.5 * max(1, args.steps + args.warmup)))
+    n_tok = max(wl.T // 8, int(wl.Lq * frac))
+    n_rows = max(1, int(8 * frac))
     for _ in range(args.warmup):
-        _oracle_sample(wl, 2)
+        sample.run(n_tok, n_rows)
     vals = []
     t0 = time.perf_counter()
-    for i in range(args.steps):
-        v, _, _ = _oracle_sample(wl, n_rows, seed=i)
-        vals.append(v)
+    for _ in range(args.steps):
+        vals.append(sample.run(n_tok, n_rows)[0])
     wall = time.perf_counter() - t0
     value = len(vals) / sum(1.0 / v for v in vals)
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    sample = (f"per step: full-chunk quantize + attention of {n_rows} query tokens x {wl.H} heads "
-              f"over {(wl.S + wl.W) * wl.T} keys")
+    desc = (f"per step: quantize of {n_tok} of the chunk's {wl.Lq} tokens x {wl.H} heads (K and V) "
+            f"+ attention of {n_rows} query tokens x {wl.H} heads over {(wl.S + wl.W) * wl.T} keys; "
+            f"tok/s = 1 / (quantize s/token + attention s/token)")
     line = {"metric": METRIC, "value": value, "unit": "query tok/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * wall / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded bf16 N(0,1), 1% K outlier channels x8)",
-            "config": {"workload": f"{wl.name}", "parallelism": "host cores"},
+            "config": bench_config(wl, args.kv, ws),
             "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": "query tok/s", "cores": cores,
-                             "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "query tok/s", "cores": _oracle_cores(),
+                             "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": "query tok/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
