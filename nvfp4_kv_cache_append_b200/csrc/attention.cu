@@ -825,39 +825,13 @@ __device__ void softmax_role(Ctx &c)
             ptx::tc_fence_after();
             const uint32_t tS = tmem + TM_S + buf * 128;
             const int nv = n_keys - tile * BN;   // valid keys of this tile (may exceed 128)
-            // pass 1: row max over the valid logits
-            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-            for (int q = 0; q < 4; ++q) {
-                float s[32];
-                ptx::tmem_ld32(tS + q * 32, reinterpret_cast<uint32_t *>(s));
-                ptx::tmem_wait_ld();
-                if (nv < BN) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (q * 32 + i >= nv) s[i] = -INFINITY;
-                }
-#pragma unroll
-                for (int i = 0; i < 32; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], s[i]);
-            }
-            const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale;
-            if (__any_sync(0xFFFFFFFFu, mt > m + 8.0f)) {
-                const float mn = fmaxf(m, mt);
-                const float alpha = ex2(m - mn);     // 0 on the first tile of a segment
-                l *= alpha;
-                m = mn;
-                if (tile > sg.t0) {
-                    // O holds the previous tile's PV once its V buffer was freed
-                    const int gp = g - 1;
-                    if (!wait_warp(c, B_VFREE + (gp & 1), (gp >> 1) & 1)) return;
-                    ptx::tc_fence_after();
-                    rescale_o(tO, alpha);
-                }
-            }
-            // pass 2: P = 2^(s * scale - m) as f16 pairs over S (keys 2i, 2i+1 ->
-            // column i); the chunk q of 32 logits becomes columns [16q, 16q + 16)
-            const float2 sc2 = make_float2(scale, scale), nm2 = make_float2(-m, -m);
+            // one pass: per chunk of 32 logits, its max first; a chunk whose
+            // max exceeds the running max m by more than 2^8 raises m (on a
+            // segment's first chunk always, rarely after), rescaling the P
+            // already written in this tile, the partial sums and O
             float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            float alpha_o = 1.0f;
+            bool grew = false;
 #pragma unroll 1
             for (int q = 0; q < 4; ++q) {
                 float s[32];
@@ -868,6 +842,36 @@ __device__ void softmax_role(Ctx &c)
                     for (int i = 0; i < 32; ++i)
                         if (q * 32 + i >= nv) s[i] = -INFINITY;
                 }
+                float mx4[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+                for (int i = 4; i < 32; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], s[i]);
+                const float cm = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale;
+                if (__any_sync(0xFFFFFFFFu, cm > m + 8.0f)) {
+                    const float mn = fmaxf(m, cm);
+                    const float al = ex2(m - mn);          // 0 while m is -inf
+                    m = mn;
+                    l *= al;
+                    alpha_o *= al;
+                    grew = true;
+                    acc[0] = __fmul2_rn(acc[0], make_float2(al, al));
+                    acc[1] = __fmul2_rn(acc[1], make_float2(al, al));
+                    if (q > 0) {
+                        ptx::tmem_wait_st();
+                        for (int k = 0; k < q; ++k) {
+                            uint32_t v[16];
+                            ptx::tmem_ld16(tS + k * 16, v);
+                            ptx::tmem_wait_ld();
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const float2 f = __half22float2(as_h2(v[i]));
+                                v[i] = pack_f16(f.x * al, f.y * al);
+                            }
+                            ptx::tmem_st16(tS + k * 16, v);
+                            ptx::tmem_wait_st();
+                        }
+                    }
+                }
+                const float2 sc2 = make_float2(scale, scale), nm2 = make_float2(-m, -m);
                 uint32_t pk[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
@@ -877,6 +881,13 @@ __device__ void softmax_role(Ctx &c)
                     pk[i] = pack_f16(p.x, p.y);
                 }
                 ptx::tmem_st16(tS + q * 16, pk);
+            }
+            if (grew && tile > sg.t0) {
+                // O holds the previous tile's PV once its V buffer was freed
+                const int gp = g - 1;
+                if (!wait_warp(c, B_VFREE + (gp & 1), (gp >> 1) & 1)) return;
+                ptx::tc_fence_after();
+                rescale_o(tO, alpha_o);
             }
             const float2 at = __fadd2_rn(acc[0], acc[1]);
             l += at.x + at.y;

@@ -79,3 +79,36 @@ def test_ragged_small_frames():
     # many frames and the last tile is ragged
     wl = kvsynth.Workload("odd", B=2, H=3, D=128, grid_h=4, grid_w=5, C=2, S=2, W=6, steps=6)
     _run(wl, 0, {1, 4, 6}, lambda wl, s, b, h: np.arange(wl.Lq), lambda wl, s, b: range(wl.H))
+
+
+@pytest.mark.parametrize("kv_dtype", [0, 1], ids=["nvfp4", "bf16"])
+def test_growing_logits_rescale(kv_dtype):
+    """Keys of later frames grow step by step (x3 .. x6; the sink's chunk
+    sets amax = 64 so that nothing saturates), so their logits sit more than
+    2^8 above the sink's: the online softmax raises its running max between
+    tiles and, with 192 tokens per frame, inside a tile that starts in the
+    sink and ends in the window (P already written and O rescaled), and must
+    still match the oracle on every row.  16 heads make 160 key tiles, so the
+    persistent schedule gives each CTA pair segments of several tiles and the
+    rescale of O between tiles runs too."""
+    wl = kvsynth.Workload("grow", B=1, H=16, D=128, grid_h=16, grid_w=12, C=1, S=1, W=4, steps=5)
+    lib = LibStream(wl, kv_dtype)
+    ora = OracleStream(wl, seed=0, keep_inputs=True)
+    quantized = kv_dtype == 0
+    for step in range(1, wl.steps + 1):
+        x = kvsynth.chunk_qkv(wl, step, 0)
+        k = x["k"].float()
+        if step == 1:
+            k[0, 0, :, 0] = 64.0
+        else:
+            k = k * (1.0 + step)
+        k = k.to(torch.bfloat16)
+        ora.step(k=k, v=x["v"], q=x["q"])
+        g = to_gpu({"q": x["q"], "k": k, "v": x["v"]})
+        out, _ = lib.step(g["q"], g["k"], g["v"])
+        torch.cuda.synchronize()
+        assert lib.cache.device_status() == 0
+        got = out.float().cpu().numpy()
+        for h in range(wl.H):
+            ref, _ = ora.attention(0, h, np.arange(wl.Lq), quantized=quantized)
+            assert_parity(got[0, :, h], ref, f"step {step} h {h}")
