@@ -236,6 +236,26 @@ NVKV_API nvkv_status nvfp4_kv_append_noalloc(const nvkv_desc *desc, const nvkv_c
 NVKV_API nvkv_status bf16_kv_append(const nvkv_desc *desc, const nvkv_cache *cache, nvkv_ring *ring,
                            const void *k, const void *v, nvkv_stream stream);
 
+/* In-place overwrite of the newest chunk, for the denoising steps of one AR
+ * step ("NVlabs/LongLive 2.0: NVFP4 parallel infrastructure for long video
+ * generation", section "NVFP4, sequence parallel and the async decode path":
+ * in-place quantized KV-cache updates; the generator refines each chunk over
+ * 2 or 4 denoising steps, and every step recomputes that chunk's K/V).
+ * k, v: device bf16 [B][Lq][H][128], the chunk's new K/V.  Quantizes them
+ * (NVFP4) or copies them (bf16 twin) into the physical slots of every
+ * stream's C newest frames, the same slots their append used; the ring is
+ * not modified and eviction does not run.  While the first chunk is the only
+ * chunk appended (ring->steps == 1) the overwrite measures that chunk's amax
+ * again and fixes s_g from the new values; afterwards s_g stays as it is.
+ * NVKV_ERR_STATE if no chunk was appended yet or the desc and ring disagree;
+ * the other errors as for the appends. */
+NVKV_API nvkv_status nvfp4_kv_overwrite(const nvkv_desc *desc, const nvkv_cache *cache,
+                                        const nvkv_ring *ring, const void *k, const void *v,
+                                        nvkv_stream stream);
+NVKV_API nvkv_status bf16_kv_overwrite(const nvkv_desc *desc, const nvkv_cache *cache,
+                                       const nvkv_ring *ring, const void *k, const void *v,
+                                       nvkv_stream stream);
+
 /* Device workspace the attention calls need on the current device (0 for an
  * invalid desc or without a device).  The attention kernels run a persistent
  * grid of CTA pairs; query tiles cut between pairs leave partial results

@@ -6,10 +6,11 @@ as the C entry points) plus ``KVCache``, which allocates the caller-owned
 device planes with PyTorch.  Importing fails loudly if the library is absent.
 """
 from . import _lib
-from ._lib import (NVKV_KV_BF16, NVKV_KV_NVFP4, NvkvError, bf16_kv_append,
+from ._lib import (NVKV_KV_BF16, NVKV_KV_NVFP4, NvkvError, bf16_kv_append, bf16_kv_overwrite,
                    chunk_attention_bf16kv, chunk_attention_nvfp4kv, kv_ring_begin_shot,
                    kv_ring_evict, nvfp4_kv_append, nvkv_attention_workspace_bytes,
-                   nvkv_desc_init, nvkv_encode_block_scale, nvkv_encode_e2m1, nvkv_plane_bytes,
+                   nvfp4_kv_overwrite, nvkv_desc_init, nvkv_encode_block_scale, nvkv_encode_e2m1,
+                   nvkv_plane_bytes,
                    nvkv_ring_init, nvkv_ring_push_chunk, nvkv_ring_visible,
                    nvkv_status_string)
 from .cache import KVCache
@@ -17,5 +18,6 @@ from .cache import KVCache
 __all__ = ["KVCache", "NvkvError", "NVKV_KV_NVFP4", "NVKV_KV_BF16", "nvkv_desc_init",
            "nvkv_plane_bytes", "nvkv_ring_init", "kv_ring_evict", "kv_ring_begin_shot",
            "nvkv_ring_visible", "nvkv_ring_push_chunk", "nvfp4_kv_append", "bf16_kv_append",
+           "nvfp4_kv_overwrite", "bf16_kv_overwrite",
            "nvkv_attention_workspace_bytes", "chunk_attention_nvfp4kv", "chunk_attention_bf16kv",
            "nvkv_encode_e2m1", "nvkv_encode_block_scale", "nvkv_status_string"]

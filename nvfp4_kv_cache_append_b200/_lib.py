@@ -89,6 +89,8 @@ def _load():
         "nvfp4_kv_append": (i32, [D, C, R, vp, vp, vp]),
         "bf16_kv_append": (i32, [D, C, R, vp, vp, vp]),
         "nvfp4_kv_append_noalloc": (i32, [D, C, R, vp, vp, vp]),
+        "nvfp4_kv_overwrite": (i32, [D, C, R, vp, vp, vp]),
+        "bf16_kv_overwrite": (i32, [D, C, R, vp, vp, vp]),
         "nvkv_attention_workspace_bytes": (sz, [D]),
         "chunk_attention_nvfp4kv": (i32, [D, C, R, vp, vp, vp, vp, sz, vp]),
         "chunk_attention_bf16kv": (i32, [D, C, R, vp, vp, vp, vp, sz, vp]),
@@ -169,6 +171,16 @@ def nvkv_ring_push_chunk(desc: nvkv_desc, ring: nvkv_ring):
 def nvfp4_kv_append(desc, cache, ring, k_ptr, v_ptr, stream=0) -> None:
     _check(lib.nvfp4_kv_append(ctypes.byref(desc), ctypes.byref(cache), ctypes.byref(ring),
                                k_ptr, v_ptr, stream), "nvfp4_kv_append")
+
+
+def nvfp4_kv_overwrite(desc, cache, ring, k_ptr, v_ptr, stream=0) -> None:
+    _check(lib.nvfp4_kv_overwrite(ctypes.byref(desc), ctypes.byref(cache), ctypes.byref(ring),
+                                  k_ptr, v_ptr, stream), "nvfp4_kv_overwrite")
+
+
+def bf16_kv_overwrite(desc, cache, ring, k_ptr, v_ptr, stream=0) -> None:
+    _check(lib.bf16_kv_overwrite(ctypes.byref(desc), ctypes.byref(cache), ctypes.byref(ring),
+                                 k_ptr, v_ptr, stream), "bf16_kv_overwrite")
 
 
 def nvfp4_kv_append_noalloc(desc, cache, ring, k_ptr, v_ptr, stream=0) -> None:

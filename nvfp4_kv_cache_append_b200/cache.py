@@ -112,6 +112,13 @@ class KVCache:
         fn = L.nvfp4_kv_append if self.fp4 else L.bf16_kv_append
         fn(self.desc, self.cache, self.ring, _ptr(k), _ptr(v), _stream(stream))
 
+    def overwrite(self, k: torch.Tensor, v: torch.Tensor, stream=None) -> None:
+        """Denoising step: the newest chunk's K/V replaced in place (same slots)."""
+        self._check_io(k)
+        self._check_io(v)
+        fn = L.nvfp4_kv_overwrite if self.fp4 else L.bf16_kv_overwrite
+        fn(self.desc, self.cache, self.ring, _ptr(k), _ptr(v), _stream(stream))
+
     def attention(self, q: torch.Tensor, out: Optional[torch.Tensor] = None,
                   lse: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
         self._check_io(q)

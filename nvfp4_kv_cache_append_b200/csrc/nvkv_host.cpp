@@ -109,9 +109,37 @@ void commit_append(const nvkv_desc *d, nvkv_ring *r, const int32_t *slot)
     r->steps += 1;
 }
 
-nvkv_status append_common(const nvkv_desc *desc, const nvkv_cache *cache, nvkv_ring *ring,
-                          const void *k, const void *v, cudaStream_t stream, int dtype)
+// Physical slots of every stream's newest chunk (frames n_appended - C ..
+// n_appended - 1), in frame order.  False if a stream has not appended a
+// chunk yet or one of those frames is no longer resident.
+bool newest_chunk_slots(const nvkv_desc *d, const nvkv_ring *r, int32_t *slot_out)
 {
+    for (int b = 0; b < d->B; ++b) {
+        const nvkv_ring_stream &s = r->s[b];
+        const int f0 = s.n_appended - d->C;
+        if (f0 < 0) return false;
+        int found = 0;
+        for (int i = 0; i < s.n_resident; ++i) {
+            const int c = s.frame[i] - f0;
+            if (c >= 0 && c < d->C) {
+                slot_out[b * d->C + c] = s.slot[i];
+                ++found;
+            }
+        }
+        if (found != d->C) return false;
+    }
+    return true;
+}
+
+// Quantize-append into C newly assigned slots, the ring then advanced
+// (advance = the ring), or, with advance = null, in-place overwrite of the
+// newest chunk: same slots, ring unchanged; while the first chunk is the only
+// one appended, its overwrite fixes s_g again from the new values.
+nvkv_status append_common(const nvkv_desc *desc, const nvkv_cache *cache, const nvkv_ring *ring,
+                          nvkv_ring *advance, const void *k, const void *v, cudaStream_t stream,
+                          int dtype)
+{
+    const bool overwrite = advance == nullptr;
     nvkv_status st = check_desc(desc);
     if (st != NVKV_OK) return st;
     if (desc->kv_dtype != dtype) return NVKV_ERR_STATE;
@@ -125,7 +153,11 @@ nvkv_status append_common(const nvkv_desc *desc, const nvkv_cache *cache, nvkv_r
         return NVKV_ERR_ALIGNMENT;
 
     AppendLaunch a{};
-    if (!plan_slots(desc, ring, a.slot)) return NVKV_ERR_CAPACITY;
+    if (overwrite) {
+        if (ring->steps < 1 || !newest_chunk_slots(desc, ring, a.slot)) return NVKV_ERR_STATE;
+    } else if (!plan_slots(desc, ring, a.slot)) {
+        return NVKV_ERR_CAPACITY;
+    }
     a.k = k;
     a.v = v;
     a.k_data = cache->k_data;
@@ -140,11 +172,11 @@ nvkv_status append_common(const nvkv_desc *desc, const nvkv_cache *cache, nvkv_r
     a.Lq = desc->C * a.T;
     a.R = (int)rows_per_head(desc);
     a.C = desc->C;
-    a.first = ring->scales_fixed ? 0 : 1;
+    a.first = overwrite ? (ring->steps == 1 ? 1 : 0) : (ring->scales_fixed ? 0 : 1);
     cudaError_t e = (dtype == NVKV_KV_NVFP4) ? nvkv::launch_nvfp4_append(a, stream)
                                              : nvkv::launch_bf16_append(a, stream);
     if (e != cudaSuccess) return NVKV_ERR_CUDA;
-    commit_append(desc, ring, a.slot);
+    if (!overwrite) commit_append(desc, advance, a.slot);
     return NVKV_OK;
 }
 
@@ -395,13 +427,27 @@ nvkv_status nvkv_ring_push_chunk(const nvkv_desc *desc, nvkv_ring *ring, int32_t
 nvkv_status nvfp4_kv_append(const nvkv_desc *desc, const nvkv_cache *cache, nvkv_ring *ring,
                             const void *k, const void *v, nvkv_stream stream)
 {
-    return append_common(desc, cache, ring, k, v, (cudaStream_t)stream, NVKV_KV_NVFP4);
+    return append_common(desc, cache, ring, ring, k, v, (cudaStream_t)stream, NVKV_KV_NVFP4);
 }
 
 nvkv_status bf16_kv_append(const nvkv_desc *desc, const nvkv_cache *cache, nvkv_ring *ring,
                            const void *k, const void *v, nvkv_stream stream)
 {
-    return append_common(desc, cache, ring, k, v, (cudaStream_t)stream, NVKV_KV_BF16);
+    return append_common(desc, cache, ring, ring, k, v, (cudaStream_t)stream, NVKV_KV_BF16);
+}
+
+nvkv_status nvfp4_kv_overwrite(const nvkv_desc *desc, const nvkv_cache *cache,
+                               const nvkv_ring *ring, const void *k, const void *v,
+                               nvkv_stream stream)
+{
+    return append_common(desc, cache, ring, nullptr, k, v, (cudaStream_t)stream, NVKV_KV_NVFP4);
+}
+
+nvkv_status bf16_kv_overwrite(const nvkv_desc *desc, const nvkv_cache *cache,
+                              const nvkv_ring *ring, const void *k, const void *v,
+                              nvkv_stream stream)
+{
+    return append_common(desc, cache, ring, nullptr, k, v, (cudaStream_t)stream, NVKV_KV_BF16);
 }
 
 size_t nvkv_attention_workspace_bytes(const nvkv_desc *desc)

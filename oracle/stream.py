@@ -65,22 +65,51 @@ class OracleStream:
                 for fid in ring.evict(need):
                     self.store.pop((b, fid), None)
             fids = ring.append()
-            for c, fid in enumerate(fids):
-                sl = slice(c * wl.T, (c + 1) * wl.T)
-                ent = {}
-                for name, xf, t in (("k", kf, 0), ("v", vf, 1)):
-                    rows = np.ascontiguousarray(xf[b, sl].transpose(1, 0, 2))   # [H, T, D]
-                    codes = np.zeros((wl.H, wl.T, 64), np.uint8)
-                    scales = np.zeros((wl.H, wl.T, 8), np.uint8)
-                    for h in range(wl.H):
-                        codes[h], scales[h] = quantize_rows(rows[h], self.s_g[t, b, h])
-                    ent[name + "_codes"] = codes
-                    ent[name + "_scales"] = scales
-                    if self.keep_inputs:
-                        ent[name + "_bf16"] = rows
-                self.store[(b, fid)] = ent
+            self._store_chunk(b, fids, kf, vf)
             new[b] = fids
         return new
+
+    def overwrite(self, k, v, q):
+        """A denoising step inside the current AR step: the newest chunk's K/V
+        replaced in place, ring unchanged (the pages' in-place quantized
+        KV-cache update, "NVlabs/LongLive 2.0: NVFP4 parallel infrastructure
+        for long video generation", section "NVFP4, sequence parallel and the
+        async decode path").  Reading: while the first chunk is the only
+        chunk appended, its global scales are fixed again from the new
+        values, since they are defined by the first chunk; afterwards they
+        stay fixed.  Returns {b: [the chunk's frame indices]}."""
+        wl = self.wl
+        if self.step_no < 1:
+            raise ValueError("no chunk appended yet")
+        self.q = q
+        if self.step_no == 1:
+            self.s_g = self._scales_from(k, v)
+        kf = k.float().numpy()
+        vf = v.float().numpy()
+        new = {}
+        for b, ring in enumerate(self.rings):
+            fids = list(range(ring.next_fid - wl.C, ring.next_fid))
+            self._store_chunk(b, fids, kf, vf)
+            new[b] = fids
+        return new
+
+    def _store_chunk(self, b, fids, kf, vf):
+        """Quantize the chunk's frames of stream b (quantize_rows per head)."""
+        wl = self.wl
+        for c, fid in enumerate(fids):
+            sl = slice(c * wl.T, (c + 1) * wl.T)
+            ent = {}
+            for name, xf, t in (("k", kf, 0), ("v", vf, 1)):
+                rows = np.ascontiguousarray(xf[b, sl].transpose(1, 0, 2))   # [H, T, D]
+                codes = np.zeros((wl.H, wl.T, 64), np.uint8)
+                scales = np.zeros((wl.H, wl.T, 8), np.uint8)
+                for h in range(wl.H):
+                    codes[h], scales[h] = quantize_rows(rows[h], self.s_g[t, b, h])
+                ent[name + "_codes"] = codes
+                ent[name + "_scales"] = scales
+                if self.keep_inputs:
+                    ent[name + "_bf16"] = rows
+            self.store[(b, fid)] = ent
 
     # ------------------------------------------------------------- read
 

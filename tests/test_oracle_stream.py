@@ -147,3 +147,38 @@ def test_shot_lengths_recipe():
     for l in lens:
         assert sum(l) == 24 and len(l) == 3 and min(l) >= 2
     assert len({tuple(l) for l in lens}) > 1
+
+
+@pytest.mark.parametrize("at_step", [1, 3, 6])
+def test_overwrite_equals_append_of_the_new_values(at_step):
+    """A denoising overwrite leaves the oracle stream exactly as if the chunk
+    had been appended with the new values in the first place: same frames,
+    same codes and scales, the same global scales (fixed again at step 1,
+    kept afterwards) and the same attention."""
+    wl = kvsynth.WORKLOADS["tiny"]
+    a = OracleStream(wl, seed=0)
+    b = OracleStream(wl, seed=0)
+    for step in range(1, at_step + 1):
+        x = kvsynth.chunk_qkv(wl, step, 0)
+        if step < at_step:
+            a.step(k=x["k"], v=x["v"], q=x["q"])
+            b.step(k=x["k"], v=x["v"], q=x["q"])
+            continue
+        y = kvsynth.chunk_qkv(wl, step + 100, 0)       # the refined K/V of the same chunk
+        a.step(k=x["k"], v=x["v"], q=x["q"])
+        s_before = a.s_g.copy()
+        new_a = a.overwrite(k=y["k"], v=y["v"], q=y["q"])
+        new_b = b.step(k=y["k"], v=y["v"], q=y["q"])
+        assert new_a == new_b
+        if at_step > 1:
+            assert np.array_equal(a.s_g, s_before)
+    assert np.array_equal(a.s_g, b.s_g)
+    assert a.rings[0].resident() == b.rings[0].resident()
+    for fid in a.rings[0].resident():
+        ea, eb = a.frame(0, fid), b.frame(0, fid)
+        for key in ("k_codes", "k_scales", "v_codes", "v_scales"):
+            assert np.array_equal(ea[key], eb[key]), (fid, key)
+    for h in range(wl.H):
+        oa, la = a.attention(0, h, np.arange(wl.Lq))
+        ob, lb = b.attention(0, h, np.arange(wl.Lq))
+        assert np.array_equal(oa, ob) and np.array_equal(la, lb)
