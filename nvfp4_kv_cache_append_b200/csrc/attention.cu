@@ -19,10 +19,11 @@
 //   K: keys [64r, 64r+64) of the tile (all 128 channels),
 //   V: channels [64r, 64r+64) of all 128 keys   (r = CTA rank in the pair).
 // Per CTA, 16 warps:
-//   warps 0-3    softmax: thread r owns query row r = TMEM lane r.  Per tile a
-//                max pass and a probability pass over the 128 logits in TMEM,
-//                P (f16) written back over S; online softmax with lazy rescale
-//                of O (when the row max grows by more than 2^8).
+//   warps 0-3    softmax: thread r owns query row r = TMEM lane r.  Per tile
+//                one pass over the 128 logits in TMEM in chunks of 32 (the
+//                chunk's max, then its exponentials), P (f16) written back
+//                over S; online softmax with lazy rescale of O (when the row
+//                max grows by more than 2^8).
 //   warps 4-7    K converters (two threads per key) and, per work segment,
 //                the RoPE-rotated Q tile into TMEM.
 //   warps 8-11   V converters (one thread per key).
@@ -240,17 +241,21 @@ __device__ __forceinline__ void set_abort(Ctx &c)
 
 __device__ __forceinline__ bool wait(Ctx &c, int bar, uint32_t parity)
 {
-    if (ptx::mbar_wait_cluster(&c.ctl->bar[bar], parity, &c.ctl->abort, WAIT_LIMIT_NS)) return true;
+    if (ptx::mbar_wait(&c.ctl->bar[bar], parity, &c.ctl->abort, WAIT_LIMIT_NS)) return true;
     set_abort(c);
     return false;
 }
 
 // Cross-CTA events (Q ready, K/V halves converted, P written, O read) are
 // counted on the even CTA's barrier.  Every thread arrives on its own CTA's
-// copy with a CTA-scope release (a few cycles); in the odd CTA one relay
-// thread per event stream waits for the local phase and forwards it with a
-// single cluster-scope release arrive (a few hundred cycles, paid once per
-// event instead of once per thread).
+// copy; in the odd CTA one relay thread per event stream waits for the local
+// phase and forwards it with a single remote arrive.  All arrives release and
+// all waits acquire at CTA scope: what an event publishes is in the
+// publishing CTA's own shared memory (made visible to the tensor core by
+// fence.proxy.async) or TMEM (ordered by the tcgen05 thread-sync fences), and
+// the peer reads it only through the pair MMA issued after the wait.  A
+// cluster-scope release or acquire costs hundreds of cycles per event here
+// and lengthens the P -> PV -> S -> softmax loop by as much.
 __device__ __forceinline__ void arrive_x(Ctx &c, int bar) { ptx::mbar_arrive(&c.ctl->bar[bar]); }
 
 // wait by every lane of a warp, outcome made warp-uniform (the tcgen05 loads
@@ -1049,7 +1054,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         // both CTAs: every MMA touching this CTA's TMEM has completed
         const int never = 0;
         if ((threadIdx.x & 31) == 0)
-            ptx::mbar_wait_cluster(&c.ctl->bar[B_MMADONE], 0, &never, WAIT_LIMIT_NS);
+            ptx::mbar_wait(&c.ctl->bar[B_MMADONE], 0, &never, WAIT_LIMIT_NS);
         __syncwarp();
     } else if (c.rank == 1 && (threadIdx.x & 31) == 0) {
         if (warp == 14) relay_qk_role(c);

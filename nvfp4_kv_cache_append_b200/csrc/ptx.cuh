@@ -74,33 +74,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
     }
 }
 
-// Wait on a barrier that other CTAs of the cluster arrive on (acquire at
-// cluster scope); same bounds as mbar_wait.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity,
-                                                  const volatile int *abort, uint64_t limit_ns)
-{
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    while (true) {
-        if (mbar_try_wait_cluster(bar, parity)) return true;
-        if (*abort) return false;
-        if (globaltimer_ns() - t0 > limit_ns) return false;
-    }
-}
-
 // ------------------------------------------------------------------ cluster
 
 __device__ __forceinline__ uint32_t cluster_ctarank()
@@ -118,11 +91,15 @@ __device__ __forceinline__ uint32_t mapa(uint32_t local_saddr, uint32_t rank)
     return r;
 }
 
-// arrive (release at cluster scope) on a barrier given by shared::cluster address
+// arrive on a barrier given by its shared::cluster address (the peer CTA's),
+// with the default release semantics at CTA scope: the arriving thread's
+// published data lives in its own CTA's shared memory or TMEM, so nothing has
+// to be pushed further out before the arrive.  This is the form CUTLASS's
+// ClusterBarrier uses for its cross-CTA arrives; a cluster-scope release
+// costs hundreds of cycles here.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr)
 {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-                 : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 __device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v)
