@@ -86,11 +86,12 @@ typedef enum {
 } nvkv_status;
 
 #define NVKV_MAGIC 0x4E564B56u /* "NVKV" */
-#define NVKV_VERSION 1u
+#define NVKV_VERSION 2u
 #define NVKV_HEAD_DIM 128
 #define NVKV_MAX_BATCH 16
 #define NVKV_MAX_FRAMES 64     /* S + W */
 #define NVKV_MAX_CHUNK 16      /* C */
+#define NVKV_MAX_SHARDS 16     /* shard_count, and parts of one nvkv_lse_merge */
 
 enum { NVKV_KV_NVFP4 = 0, NVKV_KV_BF16 = 1 };
 
@@ -108,11 +109,15 @@ typedef struct {
     int32_t kv_dtype;     /* NVKV_KV_NVFP4 or NVKV_KV_BF16                      */
     float rope_base;      /* 10000                                             */
     int32_t rope_split[3];/* head_dim channels for (frame, h, w): 44, 42, 42    */
+    int32_t shard_rank;   /* sequence-parallel KV split (nvkv_desc_set_shard): */
+    int32_t shard_count;  /* this cache holds tokens [rank*T/count,
+                             (rank+1)*T/count) of every frame; 0 of 1 = all   */
 } nvkv_desc;
 
 /* Device planes of one cache (caller-owned; sizes from nvkv_plane_bytes).
- * R = (S + W) * T rows per (batch, head); physical frame slot p holds rows
- * [p*T, (p+1)*T).
+ * R = (S + W) * Ts rows per (batch, head), Ts = T / shard_count tokens of
+ * each frame; physical frame slot p holds rows [p*Ts, (p+1)*Ts), row p*Ts + i
+ * being token shard_rank*Ts + i of the frame in that slot.
  *   NVFP4: k_data/v_data = codes [B][H][R][64] u8, k_scales/v_scales = E4M3
  *          block scales [B][H][R][8] u8, amax [2][B][H] (float bits, K then
  *          V), s_g [2][B][H] f32.
@@ -164,6 +169,25 @@ typedef struct {
  * (B <= 16, S + W <= 64, 1 <= C <= min(W, 16), T >= 1, grid_h, grid_w < 65536). */
 NVKV_API nvkv_status nvkv_desc_init(nvkv_desc *desc, int B, int H, int grid_h, int grid_w, int C, int S,
                            int W, int kv_dtype);
+
+/* Sequence-parallel KV split ("NVlabs/LongLive 2.0: NVFP4 parallel
+ * infrastructure for long video generation", section "NVFP4, sequence
+ * parallel and the async decode path": sequence-parallel inference to cut the
+ * KV memory each GPU holds).  Makes desc describe shard `rank` of `count`
+ * caches that together hold the whole cache: shard r keeps tokens
+ * [r*T/count, (r+1)*T/count) of every frame, so each holds 1/count of the K/V
+ * and of the attention work.  The ring logic is unchanged: every shard runs
+ * the same ring (same slots, same eviction) on the same calls.
+ *  - The appends take the whole chunk's k, v ([B][C*T][H][128]) and write the
+ *    shard's tokens; the first append measures amax over the whole chunk, so
+ *    all shards fix the same s_g.
+ *  - The attention calls take the whole chunk's q and return, for every
+ *    query, the attention over the shard's keys only, with its lse; the
+ *    shards' results are combined by nvkv_lse_merge.
+ * NVKV_ERR_INVALID_ARG unless 1 <= count <= NVKV_MAX_SHARDS, 0 <= rank <
+ * count and T is a multiple of count; NVKV_ERR_UNSUPPORTED for an NVFP4
+ * desc with T/count odd.  count = 1 gives back the whole cache. */
+NVKV_API nvkv_status nvkv_desc_set_shard(nvkv_desc *desc, int rank, int count);
 
 /* Bytes the caller must allocate for one plane (NVKV_PLANE_*) of a cache of
  * this desc; 0 for planes the dtype does not use or for an invalid desc. */
@@ -286,6 +310,23 @@ NVKV_API nvkv_status chunk_attention_nvfp4kv(const nvkv_desc *desc, const nvkv_c
 NVKV_API nvkv_status chunk_attention_bf16kv(const nvkv_desc *desc, const nvkv_cache *cache,
                                    const nvkv_ring *ring, const void *q, void *out, float *lse,
                                    void *workspace, size_t workspace_bytes, nvkv_stream stream);
+
+/* Merge of the partial attentions of disjoint key sets (the shards of a
+ * sequence-parallel KV split) for query rows [q0, q1):
+ *   L = log sum_j exp(L_j),  O = sum_j exp(L_j - L) O_j,
+ * which is the softmax attention over the union of the key sets (a part
+ * whose L_j is -inf, no keys, is skipped).  o_parts, lse_parts: host arrays
+ * of n_parts device pointers, part j's out ([B][Lq][H][128] bf16) and lse
+ * ([B][H][Lq] f32) of an attention call.  They may point into another GPU's
+ * memory mapped into this process (peer access or IPC), so that one kernel
+ * does the exchange and the merge: the caller orders this call after every
+ * part is written.  out: device bf16 [B][q1-q0][H][128]; lse_out: NULL or
+ * device f32 [B][H][q1-q0].  NVKV_ERR_INVALID_ARG for n_parts outside
+ * 1..NVKV_MAX_SHARDS, a null pointer or a bad range; NVKV_ERR_ALIGNMENT
+ * unless the out pointers are 16-byte and the lse pointers 4-byte aligned. */
+NVKV_API nvkv_status nvkv_lse_merge(int n_parts, const void *const *o_parts,
+                                    const float *const *lse_parts, int B, int H, int Lq, int q0,
+                                    int q1, void *out, float *lse_out, nvkv_stream stream);
 
 /* Diagnostics: the device conversions the append kernel uses, one value per
  * element.  y, t: device f32 [n]; codes: device u8 [n].

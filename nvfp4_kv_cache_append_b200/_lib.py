@@ -13,11 +13,12 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libnvkv.so")
 
 NVKV_MAGIC = 0x4E564B56
-NVKV_VERSION = 1
+NVKV_VERSION = 2
 NVKV_HEAD_DIM = 128
 NVKV_MAX_BATCH = 16
 NVKV_MAX_FRAMES = 64
 NVKV_MAX_CHUNK = 16
+NVKV_MAX_SHARDS = 16
 NVKV_KV_NVFP4 = 0
 NVKV_KV_BF16 = 1
 NVKV_FRAME_SINK = 1
@@ -38,7 +39,8 @@ class nvkv_desc(ctypes.Structure):
                 ("B", ctypes.c_int32), ("H", ctypes.c_int32), ("D", ctypes.c_int32),
                 ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32), ("C", ctypes.c_int32),
                 ("S", ctypes.c_int32), ("W", ctypes.c_int32), ("kv_dtype", ctypes.c_int32),
-                ("rope_base", ctypes.c_float), ("rope_split", ctypes.c_int32 * 3)]
+                ("rope_base", ctypes.c_float), ("rope_split", ctypes.c_int32 * 3),
+                ("shard_rank", ctypes.c_int32), ("shard_count", ctypes.c_int32)]
 
 
 class nvkv_cache(ctypes.Structure):
@@ -80,6 +82,9 @@ def _load():
     i32p = ctypes.POINTER(ctypes.c_int32)
     sigs = {
         "nvkv_desc_init": (i32, [D, i32, i32, i32, i32, i32, i32, i32, i32]),
+        "nvkv_desc_set_shard": (i32, [D, i32, i32]),
+        "nvkv_lse_merge": (i32, [i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, i32,
+                                 i32, vp, vp, vp]),
         "nvkv_plane_bytes": (sz, [D, i32]),
         "nvkv_ring_init": (i32, [D, R]),
         "kv_ring_evict": (i32, [D, R, i32]),
@@ -127,6 +132,21 @@ def nvkv_desc_init(B, H, grid_h, grid_w, C, S, W, kv_dtype=NVKV_KV_NVFP4) -> nvk
     _check(lib.nvkv_desc_init(ctypes.byref(d), B, H, grid_h, grid_w, C, S, W, kv_dtype),
            "nvkv_desc_init")
     return d
+
+
+def nvkv_desc_set_shard(desc: nvkv_desc, rank: int, count: int) -> None:
+    _check(lib.nvkv_desc_set_shard(ctypes.byref(desc), rank, count), "nvkv_desc_set_shard")
+
+
+def nvkv_lse_merge(o_ptrs, lse_ptrs, B, H, Lq, q0, q1, out_ptr, lse_out_ptr=None, stream=0) -> None:
+    """o_ptrs, lse_ptrs: sequences of device addresses (ints) of the parts."""
+    n = len(o_ptrs)
+    if len(lse_ptrs) != n:
+        raise ValueError("one lse per part")
+    oa = (ctypes.c_void_p * max(n, 1))(*o_ptrs)
+    la = (ctypes.c_void_p * max(n, 1))(*lse_ptrs)
+    _check(lib.nvkv_lse_merge(n, oa, la, B, H, Lq, q0, q1, out_ptr, lse_out_ptr, stream),
+           "nvkv_lse_merge")
 
 
 def nvkv_plane_bytes(desc: nvkv_desc, plane: int) -> int:

@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libnvkv.so")
-SOURCES = ["nvkv_host.cpp", "append.cu", "attention.cu", "append_noalloc.cu"]
+SOURCES = ["nvkv_host.cpp", "append.cu", "attention.cu", "append_noalloc.cu", "merge.cu"]
 HEADERS = ["nvkv_internal.h", "ptx.cuh", os.path.join("..", "..", "include", "nvkv.h")]
 
 NVCC_FLAGS = [

@@ -23,11 +23,19 @@ def _stream(stream: Optional[torch.cuda.Stream]):
 
 
 class KVCache:
-    """One sink + rolling-window KV ring (NVFP4 or bf16) on one CUDA device."""
+    """One sink + rolling-window KV ring (NVFP4 or bf16) on one CUDA device.
+
+    With ``shard_count > 1`` it is shard ``shard_rank`` of a sequence-parallel
+    KV split: it holds tokens [rank*T/count, (rank+1)*T/count) of every frame,
+    takes whole chunks in ``append``/``attention`` and returns the attention
+    over its own keys (merge the shards' results with ``lse_merge``)."""
 
     def __init__(self, B: int, H: int, grid_h: int, grid_w: int, C: int, S: int, W: int,
-                 kv_dtype: int = L.NVKV_KV_NVFP4, device="cuda"):
+                 kv_dtype: int = L.NVKV_KV_NVFP4, device="cuda", shard_rank: int = 0,
+                 shard_count: int = 1):
         self.desc = L.nvkv_desc_init(B, H, grid_h, grid_w, C, S, W, kv_dtype)
+        if shard_count != 1 or shard_rank != 0:
+            L.nvkv_desc_set_shard(self.desc, shard_rank, shard_count)
         self.ring = L.nvkv_ring_init(self.desc)
         self.device = torch.device(device)
         if self.device.type != "cuda":
@@ -60,12 +68,22 @@ class KVCache:
         return self.desc.grid_h * self.desc.grid_w
 
     @property
+    def Ts(self) -> int:
+        """Cached tokens of each frame (all T unless this is a shard)."""
+        return self.T // self.desc.shard_count
+
+    @property
+    def tok_off(self) -> int:
+        """Index within the frame of the first cached token."""
+        return self.desc.shard_rank * self.Ts
+
+    @property
     def Lq(self) -> int:
         return self.desc.C * self.T
 
     @property
     def rows(self) -> int:
-        return (self.desc.S + self.desc.W) * self.T
+        return (self.desc.S + self.desc.W) * self.Ts
 
     def footprint_bytes(self) -> int:
         ts = [self.k_data, self.v_data, self.k_scales, self.v_scales, self.amax, self.s_g,
@@ -144,3 +162,42 @@ class KVCache:
                 t.shape) != (d.B, self.Lq, d.H, 128):
             raise ValueError(f"expected contiguous CUDA bf16 [{d.B}, {self.Lq}, {d.H}, 128], got "
                              f"{t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def lse_merge(o_parts, lse_parts, q0: int = 0, q1: Optional[int] = None,
+              out: Optional[torch.Tensor] = None, lse_out: Optional[torch.Tensor] = None,
+              stream=None) -> torch.Tensor:
+    """Attention over the union of disjoint key sets, from each set's result.
+
+    o_parts: bf16 [B, Lq, H, 128] tensors (the shards' attention outputs),
+    lse_parts: their f32 [B, H, Lq] lse.  Merges query rows [q0, q1) into
+    out [B, q1 - q0, H, 128] (and lse_out [B, H, q1 - q0] if given)."""
+    B, Lq, H, _ = o_parts[0].shape
+    for t in o_parts:
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(
+                t.shape) != (B, Lq, H, 128):
+            raise ValueError("every part's out must be contiguous CUDA bf16 [B, Lq, H, 128]")
+    for t in lse_parts:
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or tuple(
+                t.shape) != (B, H, Lq):
+            raise ValueError("every part's lse must be contiguous CUDA f32 [B, H, Lq]")
+    q1 = Lq if q1 is None else q1
+    if out is None:
+        out = torch.empty((B, q1 - q0, H, 128), dtype=torch.bfloat16, device=o_parts[0].device)
+    return lse_merge_ptrs([t.data_ptr() for t in o_parts], [t.data_ptr() for t in lse_parts],
+                          B, Lq, H, q0, q1, out, lse_out, stream)
+
+
+def lse_merge_ptrs(o_ptrs, lse_ptrs, B: int, Lq: int, H: int, q0: int, q1: int,
+                   out: torch.Tensor, lse_out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """lse_merge with the parts given as device addresses (ints) of bf16
+    [B, Lq, H, 128] outs and f32 [B, H, Lq] lses, e.g. other GPUs' buffers
+    mapped into this process; out: bf16 [B, q1 - q0, H, 128]."""
+    if tuple(out.shape) != (B, q1 - q0, H, 128) or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError(f"out must be contiguous bf16 [{B}, {q1 - q0}, {H}, 128]")
+    if lse_out is not None and (tuple(lse_out.shape) != (B, H, q1 - q0) or
+                                lse_out.dtype != torch.float32 or not lse_out.is_contiguous()):
+        raise ValueError(f"lse_out must be contiguous f32 [{B}, {H}, {q1 - q0}]")
+    L.nvkv_lse_merge(list(o_ptrs), list(lse_ptrs), B, H, Lq, q0, q1, _ptr(out), _ptr(lse_out),
+                     _stream(stream))
+    return out

@@ -112,12 +112,12 @@ __device__ __forceinline__ void unpack_bf16x8(uint4 a, float *x)
     }
 }
 
-// l / T for 0 <= l < 2^24 by a float reciprocal with a one-step fix-up
+// l / Ts for 0 <= l < 2^24 by a float reciprocal with a one-step fix-up
 __device__ __forceinline__ int frame_of(int l, const AppendLaunch &a)
 {
-    int f = __float2int_rz((float)l * a.inv_T);
-    if (f * a.T > l) --f;
-    else if ((f + 1) * a.T <= l) ++f;
+    int f = __float2int_rz((float)l * a.inv_Ts);
+    if (f * a.Ts > l) --f;
+    else if ((f + 1) * a.Ts <= l) ++f;
     return f;
 }
 
@@ -188,16 +188,19 @@ __device__ __forceinline__ uint32_t quantize_block(uint4 w0, uint4 w1, float sg,
 
 // blockDim = (4H, ty): threadIdx.x = h * 4 + pair (blocks 2 pair, 2 pair + 1
 // of the token-head: 64 bytes in, 16 code bytes and 2 scale bytes out),
-// threadIdx.y = token in the CTA's token group.  grid = (ceil(Lq / ty), 2B):
-// blockIdx.y = t * B + b with t = 0 for K and 1 for V.
+// threadIdx.y = token in the CTA's token group.  grid = (ceil(C Ts / ty), 2B):
+// blockIdx.y = t * B + b with t = 0 for K and 1 for V.  Row l of the grid is
+// token tok_off + l % Ts of chunk frame l / Ts (all tokens: Ts = T).
 __global__ void __launch_bounds__(512) k_nvfp4_append(const __grid_constant__ AppendLaunch a)
 {
     const int t = blockIdx.y / a.B, b = blockIdx.y - t * a.B;
     const int l = blockIdx.x * blockDim.y + threadIdx.y;
-    if (l >= a.Lq) return;
+    if (l >= a.C * a.Ts) return;
     const int h = threadIdx.x >> 2, pr = threadIdx.x & 3;
+    const int frame = frame_of(l, a), tok = l - frame * a.Ts;
+    const int src_l = frame * a.T + a.tok_off + tok;
     const uint4 *src = reinterpret_cast<const uint4 *>(t ? a.v : a.k) +
-                       (((size_t)b * a.Lq + l) * a.H + h) * 16 + pr * 4;
+                       (((size_t)b * a.Lq + src_l) * a.H + h) * 16 + pr * 4;
     const uint4 w0 = ld_stream(src), w1 = ld_stream(src + 1);
     const uint4 w2 = ld_stream(src + 2), w3 = ld_stream(src + 3);
 
@@ -213,27 +216,27 @@ __global__ void __launch_bounds__(512) k_nvfp4_append(const __grid_constant__ Ap
     const uint32_t s0 = quantize_block(w0, w1, sg, c0);
     const uint32_t s1 = quantize_block(w2, w3, sg, c1);
 
-    const int frame = frame_of(l, a), tok = l - frame * a.T;
     const int slot = a.slot[b * a.C + frame];
-    const size_t row = (size_t)(b * a.H + h) * a.R + (size_t)slot * a.T + tok;
+    const size_t row = (size_t)(b * a.H + h) * a.R + (size_t)slot * a.Ts + tok;
     *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(t ? a.v_data : a.k_data) + row * 64 + pr * 16) =
         make_uint4(c0.x, c0.y, c1.x, c1.y);
     *reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(t ? a.v_scales : a.k_scales) + row * 8 +
                                   pr * 2) = (uint16_t)(s0 | (s1 << 8));
 }
 
-// bf16 twin: blockDim = (16H, ty), one 16-byte chunk per thread.
+// bf16 twin: blockDim = (16H, ty), one 16-byte chunk per thread; rows as in
+// k_nvfp4_append.
 __global__ void __launch_bounds__(1024) k_bf16_append(const __grid_constant__ AppendLaunch a)
 {
     const int t = blockIdx.y / a.B, b = blockIdx.y - t * a.B;
     const int l = blockIdx.x * blockDim.y + threadIdx.y;
-    if (l >= a.Lq) return;
+    if (l >= a.C * a.Ts) return;
     const int h = threadIdx.x >> 4, c = threadIdx.x & 15;
+    const int frame = frame_of(l, a), tok = l - frame * a.Ts;
     const uint4 *src = reinterpret_cast<const uint4 *>(t ? a.v : a.k) +
-                       (((size_t)b * a.Lq + l) * a.H + h) * 16 + c;
-    const int frame = frame_of(l, a), tok = l - frame * a.T;
+                       (((size_t)b * a.Lq + frame * a.T + a.tok_off + tok) * a.H + h) * 16 + c;
     const int slot = a.slot[b * a.C + frame];
-    const size_t row = (size_t)(b * a.H + h) * a.R + (size_t)slot * a.T + tok;
+    const size_t row = (size_t)(b * a.H + h) * a.R + (size_t)slot * a.Ts + tok;
     reinterpret_cast<uint4 *>(t ? a.v_data : a.k_data)[row * 16 + c] = ld_stream(src);
 }
 
@@ -269,9 +272,9 @@ dim3 append_block(int H, int per_head)
 cudaError_t launch_nvfp4_append(const AppendLaunch &a_in, cudaStream_t s)
 {
     AppendLaunch a = a_in;
-    a.inv_T = 1.0f / (float)a.T;
+    a.inv_Ts = 1.0f / (float)a.Ts;
     const dim3 blk = append_block(a.H, 4);
-    const dim3 grid((a.Lq + blk.y - 1) / blk.y, 2 * a.B);
+    const dim3 grid((a.C * a.Ts + blk.y - 1) / blk.y, 2 * a.B);
     if (a.first) {
         cudaError_t e = cudaMemsetAsync(a.amax, 0, sizeof(uint32_t) * 2 * a.B * a.H, s);
         if (e != cudaSuccess) return e;
@@ -289,9 +292,9 @@ cudaError_t launch_nvfp4_append(const AppendLaunch &a_in, cudaStream_t s)
 cudaError_t launch_bf16_append(const AppendLaunch &a_in, cudaStream_t s)
 {
     AppendLaunch a = a_in;
-    a.inv_T = 1.0f / (float)a.T;
+    a.inv_Ts = 1.0f / (float)a.Ts;
     const dim3 blk = append_block(a.H, 16);
-    const dim3 grid((a.Lq + blk.y - 1) / blk.y, 2 * a.B);
+    const dim3 grid((a.C * a.Ts + blk.y - 1) / blk.y, 2 * a.B);
     k_bf16_append<<<grid, blk, 0, s>>>(a);
     return cudaGetLastError();
 }

@@ -97,7 +97,9 @@ extern "C" nvkv_status nvfp4_kv_append_noalloc(const nvkv_desc *desc, const nvkv
     a.H = desc->H;
     a.T = desc->grid_h * desc->grid_w;
     a.Lq = desc->C * a.T;
-    a.R = a.T * (desc->S + desc->W);
+    a.Ts = nvkv::shard_tokens(desc);
+    a.tok_off = nvkv::shard_first_token(desc);
+    a.R = a.Ts * (desc->S + desc->W);
     a.C = desc->C;
     a.first = first;
     if (nvkv::launch_nvfp4_append(a, (cudaStream_t)stream) != cudaSuccess) return NVKV_ERR_CUDA;

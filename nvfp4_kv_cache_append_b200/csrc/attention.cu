@@ -270,7 +270,7 @@ __device__ __forceinline__ bool wait_warp(Ctx &c, int bar, uint32_t parity)
 
 __device__ __forceinline__ int key_tiles(const AttnLaunch &a, int b)
 {
-    return (a.n_vis[b] * a.T + BN - 1) / BN;
+    return (a.n_vis[b] * a.Tk + BN - 1) / BN;
 }
 
 __device__ __forceinline__ long long total_tiles(const AttnLaunch &a)
@@ -389,18 +389,22 @@ struct KeyPos {
     size_t grow;   // global row index into the [B][H][R] planes
 };
 
-__device__ __forceinline__ KeyPos key_pos(const Ctx &c, int b, int h, int n_keys, int key)
+// tok_off: index within the frame of the cache's first token (a shard of a
+// sequence-parallel KV split), a constant 0 for a whole cache
+__device__ __forceinline__ KeyPos key_pos(const Ctx &c, int b, int h, int n_keys, int key,
+                                          int tok_off)
 {
     const AttnLaunch &a = *c.a;
     KeyPos k;
     k.valid = key < n_keys;
     const int kk = k.valid ? key : 0;
-    const int f = div_fast(kk, a.T, a.inv_T);
-    const int tok = kk - f * a.T;
+    const int f = div_fast(kk, a.Tk, a.inv_Tk);
+    const int tok = kk - f * a.Tk;
     const VisFrame vf = a.vis[b][f];
-    const int hp = div_fast(tok, a.grid_w, a.inv_grid_w);
-    k.rr = rope_rows(c, vf.rope_pos, hp, tok - hp * a.grid_w);
-    k.grow = (size_t)(b * a.H + h) * a.R + (size_t)vf.slot * a.T + tok;
+    const int ft = tok_off + tok;             // the token's index in its frame
+    const int hp = div_fast(ft, a.grid_w, a.inv_grid_w);
+    k.rr = rope_rows(c, vf.rope_pos, hp, ft - hp * a.grid_w);
+    k.grow = (size_t)(b * a.H + h) * a.R + (size_t)vf.slot * a.Tk + tok;
     return k;
 }
 
@@ -544,7 +548,7 @@ __device__ __forceinline__ void conv_v_bf16(const Ctx &c, int kk, int half, cons
 }
 
 // warps 4-7: per segment the Q tile into TMEM, then K halves of the tiles
-template <bool FP4>
+template <bool FP4, bool SHARD>
 __device__ void k_converter_role(Ctx &c)
 {
     const AttnLaunch &a = *c.a;
@@ -555,7 +559,7 @@ __device__ void k_converter_role(Ctx &c)
     int g = 0;                                 // tiles processed by this CTA
     for (int si = 0; si < c.ctl->n_seg; ++si) {
         const Segment sg = c.ctl->seg[si];
-        const int n_keys = a.n_vis[sg.b] * a.T;
+        const int n_keys = a.n_vis[sg.b] * a.Tk;
         if (si > 0 && !wait_warp(c, B_QFREE, (si - 1) & 1)) return;
         ptx::tc_fence_after();
         load_q_tmem<FP4>(c, sg.b, sg.h, (2 * sg.p + (int)c.rank) * BM + t, tmem + lane_off + TM_Q);
@@ -566,7 +570,8 @@ __device__ void k_converter_role(Ctx &c)
             const int s = g % NSTAGE, kb = g & 1;
             const uint32_t stg = c.sbase + OFF_STG + s * STG_BYTES;
             const uint32_t kdst = c.sbase + OFF_K + kb * K_TILE;
-            const KeyPos k = key_pos(c, sg.b, sg.h, n_keys, tile * BN + 64 * (int)c.rank + sr);
+            const KeyPos k = key_pos(c, sg.b, sg.h, n_keys, tile * BN + 64 * (int)c.rank + sr,
+                                     SHARD ? a.tok_off : 0);
             if (FP4 && !wait(c, B_STG_FULL + s, (g / NSTAGE) & 1)) return;
             if (g >= 2 && !wait(c, B_KFREE + kb, ((g - 2) >> 1) & 1)) return;
             if (FP4) {
@@ -584,7 +589,7 @@ __device__ void k_converter_role(Ctx &c)
 }
 
 // warps 8-11: this CTA's channel half of V for all 128 keys of each tile
-template <bool FP4>
+template <bool FP4, bool SHARD>
 __device__ void v_converter_role(Ctx &c)
 {
     const AttnLaunch &a = *c.a;
@@ -592,7 +597,7 @@ __device__ void v_converter_role(Ctx &c)
     int g = 0;
     for (int si = 0; si < c.ctl->n_seg; ++si) {
         const Segment sg = c.ctl->seg[si];
-        const int n_keys = a.n_vis[sg.b] * a.T;
+        const int n_keys = a.n_vis[sg.b] * a.Tk;
         for (int tile = sg.t0; tile < sg.t1; ++tile, ++g) {
             const int s = g % NSTAGE, vb = g & 1;
             const uint32_t stg = c.sbase + OFF_STG + s * STG_BYTES;
@@ -602,7 +607,7 @@ __device__ void v_converter_role(Ctx &c)
             if (FP4) {
                 conv_v_fp4(stg, k, (int)c.rank, tile * BN + k < n_keys, vdst);
             } else {
-                const KeyPos kp = key_pos(c, sg.b, sg.h, n_keys, tile * BN + k);
+                const KeyPos kp = key_pos(c, sg.b, sg.h, n_keys, tile * BN + k, SHARD ? a.tok_off : 0);
                 conv_v_bf16(c, k, (int)c.rank, kp, vdst);
             }
             ptx::fence_proxy_async_smem();
@@ -667,9 +672,9 @@ __device__ __forceinline__ void copy_runs(const AttnLaunch &a, int b, size_t hea
                                           uint64_t *full)
 {
     for (int k = k0; k < k1;) {
-        const int f = div_fast(k, a.T, a.inv_T), tok = k - f * a.T;
-        const int n = min(a.T - tok, k1 - k);
-        const size_t g = head_row0 + (size_t)a.vis[b][f].slot * a.T + tok;
+        const int f = div_fast(k, a.Tk, a.inv_Tk), tok = k - f * a.Tk;
+        const int n = min(a.Tk - tok, k1 - k);
+        const size_t g = head_row0 + (size_t)a.vis[b][f].slot * a.Tk + tok;
         const int t0 = k - k0;
         ptx::bulk_g2s(dst_c + t0 * 64, codes + g * 64, (uint32_t)n * 64, full);
         ptx::bulk_g2s(dst_s + t0 * 8, scales + g * 8, (uint32_t)n * 8, full);
@@ -683,7 +688,7 @@ __device__ void producer_role(Ctx &c)
     int g = 0;
     for (int si = 0; si < c.ctl->n_seg; ++si) {
         const Segment sg = c.ctl->seg[si];
-        const int n_keys = a.n_vis[sg.b] * a.T;
+        const int n_keys = a.n_vis[sg.b] * a.Tk;
         const size_t head_row0 = (size_t)(sg.b * a.H + sg.h) * a.R;
         for (int tile = sg.t0; tile < sg.t1; ++tile, ++g) {
             const int s = g % NSTAGE;
@@ -818,7 +823,7 @@ __device__ void softmax_role(Ctx &c)
     int g = 0;
     for (int si = 0; si < c.ctl->n_seg; ++si) {
         const Segment sg = c.ctl->seg[si];
-        const int n_keys = a.n_vis[sg.b] * a.T;
+        const int n_keys = a.n_vis[sg.b] * a.Tk;
         const int gi = sg.b * a.H + sg.h;
         const float sgk = FP4 ? a.s_g[gi] : 1.0f;
         const float sgv = FP4 ? a.s_g[a.B * a.H + gi] : 1.0f;
@@ -990,7 +995,9 @@ __device__ void softmax_role(Ctx &c)
 
 // ------------------------------------------------------------ kernel
 
-template <bool FP4>
+// SHARD: the cache is a shard whose first token is not token 0 of the frame;
+// a separate instantiation keeps the whole-cache kernel's code as it was
+template <bool FP4, bool SHARD>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     k_chunk_attn(const __grid_constant__ AttnLaunch a)
 {
@@ -1040,9 +1047,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     if (warp < 4) {
         softmax_role<FP4>(c);
     } else if (warp < 8) {
-        k_converter_role<FP4>(c);
+        k_converter_role<FP4, SHARD>(c);
     } else if (warp < 12) {
-        v_converter_role<FP4>(c);
+        v_converter_role<FP4, SHARD>(c);
     } else if (warp == 12) {
         if (FP4 && (threadIdx.x & 31) == 0) producer_role(c);
     } else if (warp == 13) {
@@ -1069,18 +1076,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     }
 }
 
-template <bool FP4>
+template <bool FP4, bool SHARD>
 cudaError_t launch(const AttnLaunch &a, cudaStream_t s)
 {
     const uint32_t tab =
         (uint32_t)(a.n_fpos * PAIRS_F + a.grid_h * PAIRS_H + a.grid_w * PAIRS_W) * 8;
     const uint32_t bytes = 1024 + OFF_TAB + ((tab + 63) & ~63u) + sizeof(SharedCtl);
     if (bytes > 232448) return cudaErrorInvalidConfiguration;
-    cudaError_t e = cudaFuncSetAttribute(k_chunk_attn<FP4>,
+    cudaError_t e = cudaFuncSetAttribute(k_chunk_attn<FP4, SHARD>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
     const dim3 grid(2 * a.n_slots, 1, 1);
-    k_chunk_attn<FP4><<<grid, NTHREADS, bytes, s>>>(a);
+    k_chunk_attn<FP4, SHARD><<<grid, NTHREADS, bytes, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -1102,7 +1109,9 @@ int attention_slots(int device)
 
 cudaError_t launch_chunk_attention(const AttnLaunch &a, cudaStream_t s)
 {
-    return a.kv_dtype == NVKV_KV_NVFP4 ? launch<true>(a, s) : launch<false>(a, s);
+    if (a.tok_off)
+        return a.kv_dtype == NVKV_KV_NVFP4 ? launch<true, true>(a, s) : launch<false, true>(a, s);
+    return a.kv_dtype == NVKV_KV_NVFP4 ? launch<true, false>(a, s) : launch<false, false>(a, s);
 }
 
 }  // namespace nvkv

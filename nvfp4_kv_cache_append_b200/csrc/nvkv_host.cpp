@@ -47,7 +47,10 @@ nvkv_status check_desc(const nvkv_desc *d)
         d->rope_split[1] < 0 || d->rope_split[2] < 0 || !(d->rope_base > 0.0f))
         return NVKV_ERR_INVALID_ARG;
     const int64_t T = (int64_t)d->grid_h * d->grid_w;
-    const int64_t R = T * (d->S + d->W);
+    if (d->shard_count < 1 || d->shard_count > NVKV_MAX_SHARDS || d->shard_rank < 0 ||
+        d->shard_rank >= d->shard_count || T % d->shard_count)
+        return NVKV_ERR_INVALID_ARG;
+    const int64_t R = T / d->shard_count * (d->S + d->W);
     // 32-bit index arithmetic in the kernels
     if (R * d->B * d->H * 128 >= (int64_t(1) << 31) / 2 ||
         T * d->C * d->B * d->H * 128 >= (int64_t(1) << 31) / 2)
@@ -66,7 +69,7 @@ nvkv_status check_ring(const nvkv_desc *d, const nvkv_ring *r)
     return NVKV_OK;
 }
 
-int64_t rows_per_head(const nvkv_desc *d) { return (int64_t)d->grid_h * d->grid_w * (d->S + d->W); }
+int64_t rows_per_head(const nvkv_desc *d) { return (int64_t)nvkv::shard_tokens(d) * (d->S + d->W); }
 
 bool is_visible(const nvkv_ring_stream &s, int i)
 {
@@ -170,6 +173,8 @@ nvkv_status append_common(const nvkv_desc *desc, const nvkv_cache *cache, const 
     a.H = desc->H;
     a.T = desc->grid_h * desc->grid_w;
     a.Lq = desc->C * a.T;
+    a.Ts = nvkv::shard_tokens(desc);
+    a.tok_off = nvkv::shard_first_token(desc);
     a.R = (int)rows_per_head(desc);
     a.C = desc->C;
     a.first = overwrite ? (ring->steps == 1 ? 1 : 0) : (ring->scales_fixed ? 0 : 1);
@@ -235,12 +240,14 @@ nvkv_status attention_common(const nvkv_desc *desc, const nvkv_cache *cache,
     a.grid_h = desc->grid_h;
     a.inv_T = 1.0f / (float)a.T;
     a.inv_grid_w = 1.0f / (float)desc->grid_w;
+    a.Tk = nvkv::shard_tokens(desc);
+    a.tok_off = nvkv::shard_first_token(desc);
+    a.inv_Tk = 1.0f / (float)a.Tk;
     // the attention kernels are built for the 44/42/42 split and small grids;
     // the NVFP4 kernel stages scale rows with 16-byte bulk copies, which needs
-    // an even number of tokens per frame
+    // an even number of cached tokens per frame
     if (desc->rope_split[0] != 44 || desc->rope_split[1] != 42 || desc->rope_split[2] != 42 ||
-        desc->grid_h > 256 || desc->grid_w > 256 ||
-        (dtype == NVKV_KV_NVFP4 && ((desc->grid_h * desc->grid_w) & 1)))
+        desc->grid_h > 256 || desc->grid_w > 256 || (dtype == NVKV_KV_NVFP4 && (a.Tk & 1)))
         return NVKV_ERR_UNSUPPORTED;
     {
         int p = 0;
@@ -272,7 +279,7 @@ nvkv_status attention_common(const nvkv_desc *desc, const nvkv_cache *cache,
     a.n_pairs = query_pairs(desc);
     int64_t total = 0, min_tiles = INT64_MAX;
     for (int b = 0; b < desc->B; ++b) {
-        const int64_t nkt = ceil_div((int64_t)a.n_vis[b] * a.T, kTileKeys);
+        const int64_t nkt = ceil_div((int64_t)a.n_vis[b] * a.Tk, kTileKeys);
         total += (int64_t)desc->H * a.n_pairs * nkt;
         min_tiles = std::min(min_tiles, nkt);
     }
@@ -308,7 +315,22 @@ nvkv_status nvkv_desc_init(nvkv_desc *desc, int B, int H, int grid_h, int grid_w
     desc->rope_split[0] = 44;
     desc->rope_split[1] = 42;
     desc->rope_split[2] = 42;
+    desc->shard_rank = 0;
+    desc->shard_count = 1;
     return check_desc(desc);
+}
+
+nvkv_status nvkv_desc_set_shard(nvkv_desc *desc, int rank, int count)
+{
+    if (!desc) return NVKV_ERR_INVALID_ARG;
+    nvkv_desc d = *desc;
+    d.shard_rank = rank;
+    d.shard_count = count;
+    nvkv_status st = check_desc(&d);
+    if (st != NVKV_OK) return st;
+    if (d.kv_dtype == NVKV_KV_NVFP4 && (nvkv::shard_tokens(&d) & 1)) return NVKV_ERR_UNSUPPORTED;
+    *desc = d;
+    return NVKV_OK;
 }
 
 size_t nvkv_plane_bytes(const nvkv_desc *d, int plane)
@@ -459,7 +481,7 @@ size_t nvkv_attention_workspace_bytes(const nvkv_desc *desc)
     if (dev_slots < 1) return 0;
     // bound over every ring state: at most S + W visible frames, at least the
     // chunk's own C frames
-    const int64_t T = (int64_t)desc->grid_h * desc->grid_w;
+    const int64_t T = nvkv::shard_tokens(desc);
     const int64_t max_tiles = ceil_div((desc->S + desc->W) * T, kTileKeys);
     const int64_t min_tiles = ceil_div(desc->C * T, kTileKeys);
     const int64_t total = (int64_t)desc->B * desc->H * query_pairs(desc) * max_tiles;
@@ -480,6 +502,34 @@ nvkv_status chunk_attention_bf16kv(const nvkv_desc *desc, const nvkv_cache *cach
 {
     return attention_common(desc, cache, ring, q, out, lse, workspace, workspace_bytes,
                             (cudaStream_t)stream, NVKV_KV_BF16);
+}
+
+nvkv_status nvkv_lse_merge(int n_parts, const void *const *o_parts, const float *const *lse_parts,
+                           int B, int H, int Lq, int q0, int q1, void *out, float *lse_out,
+                           nvkv_stream stream)
+{
+    if (n_parts < 1 || n_parts > NVKV_MAX_SHARDS || !o_parts || !lse_parts || !out || B < 1 ||
+        H < 1 || Lq < 1 || q0 < 0 || q1 > Lq || q0 >= q1)
+        return NVKV_ERR_INVALID_ARG;
+    if ((int64_t)B * Lq * H * 128 >= (int64_t(1) << 31)) return NVKV_ERR_UNSUPPORTED;
+    nvkv::MergeLaunch m{};
+    for (int j = 0; j < n_parts; ++j) {
+        if (!o_parts[j] || !lse_parts[j]) return NVKV_ERR_INVALID_ARG;
+        if (!aligned16(o_parts[j]) || (reinterpret_cast<uintptr_t>(lse_parts[j]) & 3u))
+            return NVKV_ERR_ALIGNMENT;
+        m.o[j] = o_parts[j];
+        m.lse[j] = lse_parts[j];
+    }
+    if (!aligned16(out) || (reinterpret_cast<uintptr_t>(lse_out) & 3u)) return NVKV_ERR_ALIGNMENT;
+    m.n = n_parts;
+    m.B = B;
+    m.H = H;
+    m.Lq = Lq;
+    m.q0 = q0;
+    m.nq = q1 - q0;
+    m.out = out;
+    m.lse_out = lse_out;
+    return nvkv::launch_lse_merge(m, (cudaStream_t)stream) == cudaSuccess ? NVKV_OK : NVKV_ERR_CUDA;
 }
 
 nvkv_status nvkv_encode_e2m1(const float *y, uint8_t *codes, size_t n, nvkv_stream stream)

@@ -16,11 +16,20 @@ struct AppendLaunch {
     void *k_scales, *v_scales;       // E4M3 [B][H][R][8] (NVFP4 only)
     uint32_t *amax;                  // [2][B][H]
     float *s_g;                      // [2][B][H]
-    int B, H, T, Lq, R, C;
-    float inv_T;                     // 1/T, set by the launchers (frame index by reciprocal)
+    int B, H, T, Lq, R, C;           // T tokens per frame, Lq = C * T rows of k, v
+    int Ts, tok_off;                 // this shard's tokens of a frame: [tok_off, tok_off + Ts)
+    float inv_Ts;                    // 1/Ts, set by the launchers (frame index by reciprocal)
     int first;                       // 1: measure amax and fix s_g
     int32_t slot[NVKV_MAX_BATCH * NVKV_MAX_CHUNK];  // [b * C + c] -> physical slot
 };
+
+// Tokens per frame of the cache a desc describes (the shard's share of each
+// frame) and the index of its first token within the frame.
+inline int shard_tokens(const nvkv_desc *d)
+{
+    return d->grid_h * d->grid_w / (d->shard_count > 0 ? d->shard_count : 1);
+}
+inline int shard_first_token(const nvkv_desc *d) { return d->shard_rank * shard_tokens(d); }
 
 cudaError_t launch_nvfp4_append(const AppendLaunch &a, cudaStream_t s);
 cudaError_t launch_bf16_append(const AppendLaunch &a, cudaStream_t s);
@@ -49,6 +58,8 @@ struct AttnLaunch {
     VisFrame vis[NVKV_MAX_BATCH][NVKV_MAX_FRAMES];
     int grid_h;
     float inv_T, inv_grid_w;         // 1/T and 1/grid_w (division by reciprocal + fix-up)
+    int Tk, tok_off;                 // cached tokens per frame (the shard's), first one's index
+    float inv_Tk;                    // 1/Tk
     int n_fpos;                      // frame positions used: 0 .. n_fpos-1
     float theta[64];                 // RoPE angle per unit position of each channel pair
     void *workspace;                 // split-item partials + counters (zero on first use)
@@ -62,5 +73,16 @@ size_t attention_workspace_bytes(int n_slots);
 int attention_slots(int device);     // CTA pairs that can be resident at once
 
 cudaError_t launch_chunk_attention(const AttnLaunch &a, cudaStream_t s);
+
+// LSE-weighted merge of the partial attentions of disjoint key sets.
+struct MergeLaunch {
+    const void *o[NVKV_MAX_SHARDS];     // bf16 [B][Lq][H][128] per part
+    const float *lse[NVKV_MAX_SHARDS];  // f32 [B][H][Lq] per part
+    int n, B, H, Lq, q0, nq;
+    void *out;                          // bf16 [B][nq][H][128]
+    float *lse_out;                     // f32 [B][H][nq] or null
+};
+
+cudaError_t launch_lse_merge(const MergeLaunch &m, cudaStream_t s);
 
 }  // namespace nvkv

@@ -116,23 +116,28 @@ class OracleStream:
     def frame(self, b: int, fid: int) -> dict:
         return self.store[(b, fid)]
 
-    def visible_kv(self, b: int, h: int, quantized: bool = True):
+    def visible_kv(self, b: int, h: int, quantized: bool = True, tokens=None):
         """Visible keys/values of the newest chunk for (b, h) in logical order.
 
         Returns (k [Lk,128] f64, v [Lk,128] f64, k_frame_pos [Lk], k_tok [Lk]).
-        ``quantized=False`` gives the bf16 cache (the bf16-KV twin)."""
+        ``quantized=False`` gives the bf16 cache (the bf16-KV twin);
+        ``tokens=(t0, t1)`` keeps tokens t0 .. t1-1 of every frame (one shard
+        of a sequence-parallel KV split, ``oracle.merge``)."""
         wl = self.wl
+        t0, t1 = (0, wl.T) if tokens is None else tokens
         ks, vs, fpos, tok = [], [], [], []
         for fid, rank in self.rings[b].visible():
             e = self.store[(b, fid)]
             if quantized:
-                ks.append(dequant_rows(e["k_codes"][h], e["k_scales"][h], self.s_g[0, b, h]))
-                vs.append(dequant_rows(e["v_codes"][h], e["v_scales"][h], self.s_g[1, b, h]))
+                ks.append(dequant_rows(e["k_codes"][h][t0:t1], e["k_scales"][h][t0:t1],
+                                       self.s_g[0, b, h]))
+                vs.append(dequant_rows(e["v_codes"][h][t0:t1], e["v_scales"][h][t0:t1],
+                                       self.s_g[1, b, h]))
             else:
-                ks.append(e["k_bf16"][h].astype(np.float64))
-                vs.append(e["v_bf16"][h].astype(np.float64))
-            fpos.append(np.full(wl.T, rank, np.int32))
-            tok.append(np.arange(wl.T, dtype=np.int32))
+                ks.append(e["k_bf16"][h][t0:t1].astype(np.float64))
+                vs.append(e["v_bf16"][h][t0:t1].astype(np.float64))
+            fpos.append(np.full(t1 - t0, rank, np.int32))
+            tok.append(np.arange(t0, t1, dtype=np.int32))
         if not ks:
             z = np.zeros((0, 128))
             return z, z, np.zeros(0, np.int32), np.zeros(0, np.int32)
@@ -143,9 +148,10 @@ class OracleStream:
         l = np.arange(wl.Lq)
         return (self.rings[b].query_pos0() + l // wl.T).astype(np.int32), (l % wl.T).astype(np.int32)
 
-    def attention(self, b: int, h: int, rows, quantized: bool = True):
-        """Oracle outputs (fp64) for query rows ``rows`` of (b, h) at the current step."""
-        k, v, fpos, tok = self.visible_kv(b, h, quantized)
+    def attention(self, b: int, h: int, rows, quantized: bool = True, tokens=None):
+        """Oracle outputs (fp64) for query rows ``rows`` of (b, h) at the current
+        step: (out [n, 128], lse [n]); ``tokens`` as in ``visible_kv``."""
+        k, v, fpos, tok = self.visible_kv(b, h, quantized, tokens)
         qpos, qtok = self.query_positions(b)
         q = self.q[b, :, h, :]
         return attention_rows(q, k, v, fpos, tok, qpos, qtok, rows, self.wl.grid_w)

@@ -40,7 +40,7 @@ def test_binding_covers_every_entry_point():
 
 
 def test_struct_sizes_match_header_layout():
-    assert ctypes.sizeof(L.nvkv_desc) == 4 * 15
+    assert ctypes.sizeof(L.nvkv_desc) == 4 * 17
     assert ctypes.sizeof(L.nvkv_cache) == 7 * 8
     assert ctypes.sizeof(L.nvkv_ring_stream) == 16 + 4 * 4 * 64
     assert ctypes.sizeof(L.nvkv_ring) == 32 + 16 * ctypes.sizeof(L.nvkv_ring_stream)
@@ -70,6 +70,41 @@ def test_desc_validation():
     assert L.lib.nvkv_ring_init(ctypes.byref(bad), ctypes.byref(L.nvkv_ring())) == 5
 
 
+def test_shard_validation():
+    d = nv.nvkv_desc_init(1, 12, 30, 52, 3, 3, 18)
+    assert (d.shard_rank, d.shard_count) == (0, 1)
+    nv.nvkv_desc_set_shard(d, 3, 4)
+    assert (d.shard_rank, d.shard_count) == (3, 4)
+    for rank, count, want in [(2, 2, "NVKV_ERR_INVALID_ARG"), (0, 0, "NVKV_ERR_INVALID_ARG"),
+                              (0, 17, "NVKV_ERR_INVALID_ARG"), (-1, 2, "NVKV_ERR_INVALID_ARG"),
+                              (0, 7, "NVKV_ERR_INVALID_ARG"),      # 1560 tokens do not split in 7
+                              (0, 8, "NVKV_ERR_UNSUPPORTED")]:     # 195 tokens: odd for NVFP4
+        e = nv.nvkv_desc_init(1, 12, 30, 52, 3, 3, 18)
+        assert _status(nv.nvkv_desc_set_shard, e, rank, count) == want, (rank, count)
+        assert (e.shard_rank, e.shard_count) == (0, 1)            # unchanged on error
+    t = nv.nvkv_desc_init(1, 12, 30, 52, 3, 3, 18, nv.NVKV_KV_BF16)
+    nv.nvkv_desc_set_shard(t, 7, 8)                                # the bf16 twin takes odd shares
+    nv.nvkv_desc_set_shard(t, 0, 1)
+    assert (t.shard_rank, t.shard_count) == (0, 1)
+
+
+def test_merge_validation_before_launch():
+    fake = 1 << 20                                                 # never dereferenced
+    for args, want in [((0, [], [], 1, 2, 8, 0, 8, fake), "NVKV_ERR_INVALID_ARG"),
+                       ((17, [fake] * 17, [fake] * 17, 1, 2, 8, 0, 8, fake), "NVKV_ERR_INVALID_ARG"),
+                       ((1, [fake], [fake], 1, 2, 8, 4, 4, fake), "NVKV_ERR_INVALID_ARG"),
+                       ((1, [fake], [fake], 1, 2, 8, 0, 9, fake), "NVKV_ERR_INVALID_ARG"),
+                       ((1, [0], [fake], 1, 2, 8, 0, 8, fake), "NVKV_ERR_INVALID_ARG"),
+                       ((1, [fake + 8], [fake], 1, 2, 8, 0, 8, fake), "NVKV_ERR_ALIGNMENT"),
+                       ((1, [fake], [fake + 2], 1, 2, 8, 0, 8, fake), "NVKV_ERR_ALIGNMENT"),
+                       ((1, [fake], [fake], 1, 2, 8, 0, 8, fake + 4), "NVKV_ERR_ALIGNMENT")]:
+        n, o, l = args[0], args[1], args[2]
+        oa = (ctypes.c_void_p * max(n, 1))(*o)
+        la = (ctypes.c_void_p * max(n, 1))(*l)
+        st = L.lib.nvkv_lse_merge(n, oa, la, *args[3:], None, None)
+        assert L.STATUS[st] == want, (args, L.STATUS[st])
+
+
 def test_plane_bytes():
     d = nv.nvkv_desc_init(1, 12, 30, 52, 3, 3, 18)
     rows = 12 * 21 * 1560
@@ -79,6 +114,10 @@ def test_plane_bytes():
     t = nv.nvkv_desc_init(1, 12, 30, 52, 3, 3, 18, nv.NVKV_KV_BF16)
     assert nv.nvkv_plane_bytes(t, L.NVKV_PLANE_K_DATA) == rows * 256
     assert nv.nvkv_plane_bytes(t, L.NVKV_PLANE_K_SCALES) == 0
+    nv.nvkv_desc_set_shard(d, 1, 4)                        # a quarter of every frame
+    assert nv.nvkv_plane_bytes(d, L.NVKV_PLANE_K_DATA) == rows // 4 * 64
+    assert nv.nvkv_plane_bytes(d, L.NVKV_PLANE_V_SCALES) == rows // 4 * 8 + 16
+    assert nv.nvkv_plane_bytes(d, L.NVKV_PLANE_SCALE_G) == 2 * 12 * 4
 
 
 def _drive(desc, ring, sched_b, step):
