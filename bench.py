@@ -345,6 +345,95 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------- sequence-parallel mode
+
+def run_sp(args):
+    """--sp: one cache split over the ranks (strong scaling).  Each rank holds
+    1/N of every frame's tokens; one step is append + attention over the
+    shard + one barrier + the merge of the rank's query slice, which reads
+    every rank's partial result (peers' over NVLink)."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import kvsynth
+    import nvfp4_kv_cache_append_b200 as nv
+    from nvfp4_kv_cache_append_b200.sp import SequenceParallelKV
+
+    ws, rank, local = _dist_env()
+    torch.cuda.set_device(local)
+    if "MASTER_ADDR" not in os.environ:          # one process without torchrun
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(29500 + os.getpid() % 1000),
+                          RANK="0", WORLD_SIZE="1")
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    wl = kvsynth.WORKLOADS[args.workload]
+    kvd = nv.NVKV_KV_NVFP4 if args.kv == "nvfp4" else nv.NVKV_KV_BF16
+    stream = torch.cuda.Stream()
+    torch.cuda.set_stream(stream)
+    n_layers = 1 if wl.name == "long600" else N_LAYERS
+    sets = [{k: v.cuda() for k, v in kvsynth.chunk_qkv(wl, 1000 + i, seed=0).items()}
+            for i in range(N_LAYERS)]
+    sps = [SequenceParallelKV(wl.B, wl.H, wl.grid_h, wl.grid_w, wl.C, wl.S, wl.W, kvd)
+           for _ in range(n_layers)]
+    q0, q1 = sps[0].plan.queries
+    outs = [torch.empty(wl.B, q1 - q0, wl.H, 128, dtype=torch.bfloat16, device="cuda")
+            for _ in range(n_layers)]
+    for li in range(n_layers):
+        for s_ in range((wl.S + wl.W) // wl.C):
+            x = sets[s_ % N_LAYERS]
+            sps[li].step(x["q"], x["k"], x["v"], out=outs[li])
+    torch.cuda.synchronize()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def one_step(i):
+        x = sets[(i + 1) % N_LAYERS]
+        sps[i % n_layers].step(x["q"], x["k"], x["v"], out=outs[i % n_layers])
+
+    for i in range(args.warmup):
+        one_step(i)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    dist.barrier()
+    a, b = ev(), ev()
+    a.record(stream)
+    for i in range(args.steps):
+        one_step(args.warmup + i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clk = clocks.stop()
+    t = torch.tensor([a.elapsed_time(b)], device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    for sp in sps:
+        assert sp.cache.device_status() == 0, "device-side pipeline error"
+    K = args.steps
+    line = {
+        "metric": METRIC, "value": wl.B * wl.Lq * K / (total_ms / 1e3), "unit": "query tok/s",
+        "n_gpus": ws, "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": "e2m1/e4m3 cache, f16 MMA, f32 accumulate" if kvd == nv.NVKV_KV_NVFP4
+                 else "bf16 MMA, f32 accumulate",
+        "data": "synthetic (seeded bf16 N(0,1), 1% K outlier channels x8)",
+        "config": dict(bench_config(wl, args.kv, ws),
+                       parallelism=f"sequence-parallel KV split x{ws}",
+                       kv_tokens_per_rank=f"{wl.T // ws} of {wl.T} per frame"),
+        "gpu_launches": 3 * K,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del sps
+    dist.barrier()
+    dist.destroy_process_group()
+
+
 # ------------------------------------------------------------ oracle arm
 
 class OracleSample:
@@ -466,11 +555,15 @@ def main():
     ap.add_argument("--kv", default="nvfp4", choices=["nvfp4", "bf16"])
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sp", action="store_true",
+                    help="sequence-parallel KV split over the ranks instead of replicas")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.sp:
+        run_sp(args)
     else:
         run_ours(args)
 

@@ -141,3 +141,39 @@ def test_merge_rejects_bad_arguments():
         L.nvkv_lse_merge([o.data_ptr() + 2], [l.data_ptr()], 1, 2, 8, 0, 8, out.data_ptr())
     with pytest.raises(ValueError):
         nv.lse_merge([o], [l], 0, 8, out=torch.empty(1, 4, 2, 128, dtype=torch.bfloat16, device="cuda"))
+
+
+def test_sequence_parallel_class_on_one_rank():
+    """SequenceParallelKV through a one-rank NCCL group: symmetric buffer,
+    barrier and the merge over the peer-pointer list; with one shard the
+    merge returns the attention output unchanged."""
+    import os
+    import socket
+
+    import torch.distributed as dist
+
+    import nvfp4_kv_cache_append_b200 as nv
+    from nvfp4_kv_cache_append_b200.sp import SequenceParallelKV
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    torch.cuda.set_device(0)
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        wl = kvsynth.WORKLOADS["tiny"]
+        sp = SequenceParallelKV(wl.B, wl.H, wl.grid_h, wl.grid_w, wl.C, wl.S, wl.W, nv.NVKV_KV_NVFP4)
+        ref = nv.KVCache(wl.B, wl.H, wl.grid_h, wl.grid_w, wl.C, wl.S, wl.W, nv.NVKV_KV_NVFP4)
+        assert sp.plan.queries == (0, wl.Lq) and len(sp.ptrs) == 1
+        for step in range(1, wl.steps + 1):
+            g = to_gpu(kvsynth.chunk_qkv(wl, step, 5))
+            got = sp.step(g["q"], g["k"], g["v"])
+            want = ref.step(g["q"], g["k"], g["v"])
+            torch.cuda.synchronize()
+            assert torch.equal(got, want), step
+        assert sp.cache.device_status() == 0
+        del sp
+    finally:
+        dist.destroy_process_group()
