@@ -256,39 +256,52 @@ def run_ours(args):
     for c in caches:
         assert c.device_status() == 0, "device-side pipeline error"
 
-    # end to end through the same calls with host buffers: pinned H2D of the
-    # step's q/k/v, the step, D2H of the output
+    # end to end through the public host pipeline: every step uploads its
+    # q/k/v from pinned host memory, runs evict + append + attention and
+    # downloads the output to pinned host memory, on three streams so that
+    # step k's upload overlaps step k-1's compute and step k-2's download
     host = [{k: v.cpu().pin_memory() for k, v in s.items()} for s in sets]
-    host_out = torch.empty(sets[0]["q"].shape, dtype=torch.bfloat16).pin_memory()
-    dev_in = {k: torch.empty_like(v) for k, v in sets[0].items()}
+    host_out = [torch.empty(sets[0]["q"].shape, dtype=torch.bfloat16).pin_memory()
+                for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host[0].values())
-    d2h = host_out.numel() * host_out.element_size()
+    d2h = host_out[0].numel() * host_out[0].element_size()
+    # one set of streams for all emulated layers: their steps run in order,
+    # as a model's layers would
+    pstreams = tuple(torch.cuda.Stream() for _ in range(3))
+    pipes = [nv.HostPipeline(c, streams=pstreams) for c in caches]
 
     def e2e_step(i):
         li = i % n_layers
-        for k, v in host[(i + 1) % N_LAYERS].items():
-            dev_in[k].copy_(v, non_blocking=True)
-        c = begin_step(li)
-        c.append(dev_in["k"], dev_in["v"], stream=stream)
-        c.attention(dev_in["q"], out=outs[li], stream=stream)
-        host_out.copy_(outs[li], non_blocking=True)
+        if sched is not None:
+            n = len(sched[0])
+            k, rep = steps_done[li] % n, steps_done[li] // n
+            shot = [sched[b][k] + wl.shots * rep for b in range(wl.B)]
+        else:
+            shot = None
+        steps_done[li] += 1
+        x = host[(i + 1) % N_LAYERS]
+        pipes[li].submit(x["q"], x["k"], x["v"], host_out[i & 1], shot=shot)
 
     for i in range(3):
         e2e_step(i)
+    for p in pipes:
+        p.synchronize()
     torch.cuda.synchronize()
     if ws > 1:
         dist.barrier()
     a, b = ev(), ev()
-    a.record(stream)
+    a.record(pstreams[0])
     for i in range(args.steps):
         e2e_step(i)
-    b.record(stream)
+    b.record(pstreams[2])
     torch.cuda.synchronize()
     e2e_ms = a.elapsed_time(b)
     if ws > 1:
         t = torch.tensor([e2e_ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
+    for c in caches:
+        assert c.device_status() == 0, "device-side pipeline error"
 
     peaks = _peaks()
     K = args.steps

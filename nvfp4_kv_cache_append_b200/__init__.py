@@ -14,8 +14,9 @@ from ._lib import (NVKV_KV_BF16, NVKV_KV_NVFP4, NvkvError, bf16_kv_append, bf16_
                    nvkv_ring_init, nvkv_ring_push_chunk, nvkv_ring_visible,
                    nvkv_status_string)
 from .cache import KVCache, lse_merge, lse_merge_ptrs
+from .pipeline import HostPipeline
 
-__all__ = ["KVCache", "lse_merge", "lse_merge_ptrs", "NvkvError", "NVKV_KV_NVFP4", "NVKV_KV_BF16",
+__all__ = ["KVCache", "HostPipeline", "lse_merge", "lse_merge_ptrs", "NvkvError", "NVKV_KV_NVFP4", "NVKV_KV_BF16",
            "nvkv_desc_init", "nvkv_desc_set_shard", "nvkv_lse_merge",
            "nvkv_plane_bytes", "nvkv_ring_init", "kv_ring_evict", "kv_ring_begin_shot",
            "nvkv_ring_visible", "nvkv_ring_push_chunk", "nvfp4_kv_append", "bf16_kv_append",
