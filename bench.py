@@ -340,7 +340,7 @@ def run_ours(args):
         "append_ms": app_avg,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak,
                      "unit": "TFLOP/s", "frac": attn_tflops / peak,
-                     "traffic": _ncu_traffic("k_chunk_attn<1>") if fp4 else None,
+                     "traffic": _ncu_traffic("k_chunk_attn<1, 0>") if fp4 else None,
                      "kernel": "k_chunk_attn", "peak_source": peaks["source"] + " bf16 (f16 same nominal rate)"},
         "append_roofline": {"bound": "hbm", "achieved": append_gbs, "peak": peaks["hbm_gbs"],
                             "unit": "GB/s", "frac": append_gbs / peaks["hbm_gbs"]},
