@@ -311,6 +311,36 @@ NVKV_API nvkv_status chunk_attention_bf16kv(const nvkv_desc *desc, const nvkv_ca
                                    const nvkv_ring *ring, const void *q, void *out, float *lse,
                                    void *workspace, size_t workspace_bytes, nvkv_stream stream);
 
+/* The K/V projection of a chunk, the step before the append, on the tensor
+ * cores: K = x W_k^T, V = x W_v^T with bf16 inputs and f32 accumulation,
+ * rounded to bf16 (round to nearest even).  x: device bf16 [B][Lq][hidden]
+ * (the chunk's hidden states, token-major), w_k, w_v: device bf16
+ * [H*128][hidden] (output channel h*128 + d in row h*128 + d), k_out, v_out:
+ * device bf16 [B][Lq][H][128].  status: device int32, cleared by the caller,
+ * receives NVKV_ERR_TIMEOUT if a pipeline wait runs out.  hidden must be a
+ * positive multiple of 64 (else NVKV_ERR_UNSUPPORTED); the desc must be a
+ * whole cache (shard_count 1).  All pointers 16-byte aligned. */
+NVKV_API nvkv_status nvkv_kv_project(const nvkv_desc *desc, const void *x, int hidden,
+                                     const void *w_k, const void *w_v, void *k_out, void *v_out,
+                                     int32_t *status, nvkv_stream stream);
+
+/* The projection with the quantize-append fused into its epilogue ("NVlabs/
+ * LongLive 2.0: NVFP4 parallel infrastructure for long video generation",
+ * section "NVFP4, sequence parallel and the async decode path": in-place
+ * quantized KV-cache updates): each token-head row of K and V is rounded to
+ * bf16 as nvkv_kv_project would return it and quantized to NVFP4 straight
+ * into the ring slot nvfp4_kv_append would give it; the bf16 K/V never
+ * reaches memory.  The result is exactly nvkv_kv_project followed by
+ * nvfp4_kv_append.  The first append of a cache fixes s_g from the whole
+ * chunk's amax, which the epilogue cannot know: it runs nvkv_kv_project into
+ * scratch (device, >= 2 * B * Lq * H * 128 * 2 bytes, else NVKV_ERR_CAPACITY)
+ * and then nvfp4_kv_append; later appends need no scratch (may be NULL).
+ * Ring update and errors as nvfp4_kv_append, and as nvkv_kv_project. */
+NVKV_API nvkv_status nvfp4_kv_project_append(const nvkv_desc *desc, const nvkv_cache *cache,
+                                             nvkv_ring *ring, const void *x, int hidden,
+                                             const void *w_k, const void *w_v, void *scratch,
+                                             size_t scratch_bytes, nvkv_stream stream);
+
 /* Merge of the partial attentions of disjoint key sets (the shards of a
  * sequence-parallel KV split) for query rows [q0, q1):
  *   L = log sum_j exp(L_j),  O = sum_j exp(L_j - L) O_j,

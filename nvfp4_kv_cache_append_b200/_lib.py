@@ -83,6 +83,8 @@ def _load():
     sigs = {
         "nvkv_desc_init": (i32, [D, i32, i32, i32, i32, i32, i32, i32, i32]),
         "nvkv_desc_set_shard": (i32, [D, i32, i32]),
+        "nvkv_kv_project": (i32, [D, vp, i32, vp, vp, vp, vp, vp, vp]),
+        "nvfp4_kv_project_append": (i32, [D, C, R, vp, i32, vp, vp, vp, sz, vp]),
         "nvkv_lse_merge": (i32, [i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, i32,
                                  i32, vp, vp, vp]),
         "nvkv_plane_bytes": (sz, [D, i32]),
@@ -147,6 +149,19 @@ def nvkv_lse_merge(o_ptrs, lse_ptrs, B, H, Lq, q0, q1, out_ptr, lse_out_ptr=None
     la = (ctypes.c_void_p * max(n, 1))(*lse_ptrs)
     _check(lib.nvkv_lse_merge(n, oa, la, B, H, Lq, q0, q1, out_ptr, lse_out_ptr, stream),
            "nvkv_lse_merge")
+
+
+def nvkv_kv_project(desc, x_ptr, hidden, wk_ptr, wv_ptr, k_out_ptr, v_out_ptr, status_ptr,
+                    stream=0) -> None:
+    _check(lib.nvkv_kv_project(ctypes.byref(desc), x_ptr, hidden, wk_ptr, wv_ptr, k_out_ptr,
+                               v_out_ptr, status_ptr, stream), "nvkv_kv_project")
+
+
+def nvfp4_kv_project_append(desc, cache, ring, x_ptr, hidden, wk_ptr, wv_ptr, scratch_ptr,
+                            scratch_bytes, stream=0) -> None:
+    _check(lib.nvfp4_kv_project_append(ctypes.byref(desc), ctypes.byref(cache), ctypes.byref(ring),
+                                       x_ptr, hidden, wk_ptr, wv_ptr, scratch_ptr, scratch_bytes,
+                                       stream), "nvfp4_kv_project_append")
 
 
 def nvkv_plane_bytes(desc: nvkv_desc, plane: int) -> int:

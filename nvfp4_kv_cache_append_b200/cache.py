@@ -137,6 +137,47 @@ class KVCache:
         fn = L.nvfp4_kv_overwrite if self.fp4 else L.bf16_kv_overwrite
         fn(self.desc, self.cache, self.ring, _ptr(k), _ptr(v), _stream(stream))
 
+    def project(self, x: torch.Tensor, w_k: torch.Tensor, w_v: torch.Tensor, k_out=None,
+                v_out=None, stream=None):
+        """K/V projection on the tensor cores: (x W_k^T, x W_v^T) rounded to
+        bf16.  x: bf16 [B, C*T, hidden]; w_k, w_v: bf16 [H*128, hidden]."""
+        hidden = self._check_proj(x, w_k, w_v)
+        k_out = torch.empty((self.desc.B, self.Lq, self.desc.H, 128), dtype=torch.bfloat16,
+                            device=x.device) if k_out is None else k_out
+        v_out = torch.empty_like(k_out) if v_out is None else v_out
+        self._check_io(k_out)
+        self._check_io(v_out)
+        L.nvkv_kv_project(self.desc, _ptr(x), hidden, _ptr(w_k), _ptr(w_v), _ptr(k_out),
+                          _ptr(v_out), _ptr(self.status), _stream(stream))
+        return k_out, v_out
+
+    def project_append(self, x: torch.Tensor, w_k: torch.Tensor, w_v: torch.Tensor,
+                       stream=None) -> None:
+        """Projection with the NVFP4 quantize-append fused into its epilogue
+        (the same cache contents as project + append)."""
+        if not self.fp4:
+            raise ValueError("the fused projection-append writes an NVFP4 cache")
+        hidden = self._check_proj(x, w_k, w_v)
+        scratch, nbytes = None, 0
+        if not self.ring.scales_fixed:
+            nbytes = 2 * self.desc.B * self.Lq * self.desc.H * 128 * 2
+            scratch = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+        L.nvfp4_kv_project_append(self.desc, self.cache, self.ring, _ptr(x), hidden, _ptr(w_k),
+                                  _ptr(w_v), _ptr(scratch), nbytes, _stream(stream))
+
+    def _check_proj(self, x, w_k, w_v) -> int:
+        d = self.desc
+        if x.dim() != 3 or tuple(x.shape[:2]) != (d.B, self.Lq):
+            raise ValueError(f"x must be [{d.B}, {self.Lq}, hidden]")
+        hidden = x.shape[2]
+        for t in (x, w_k, w_v):
+            if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+                raise ValueError("x, w_k, w_v must be contiguous CUDA bf16 tensors")
+        for w in (w_k, w_v):
+            if tuple(w.shape) != (d.H * 128, hidden):
+                raise ValueError(f"weights must be [{d.H * 128}, {hidden}]")
+        return hidden
+
     def attention(self, q: torch.Tensor, out: Optional[torch.Tensor] = None,
                   lse: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
         self._check_io(q)

@@ -504,6 +504,102 @@ nvkv_status chunk_attention_bf16kv(const nvkv_desc *desc, const nvkv_cache *cach
                             (cudaStream_t)stream, NVKV_KV_BF16);
 }
 
+namespace {
+
+nvkv_status check_project(const nvkv_desc *desc, const void *x, int hidden, const void *w_k,
+                          const void *w_v)
+{
+    nvkv_status st = check_desc(desc);
+    if (st != NVKV_OK) return st;
+    if (!x || !w_k || !w_v) return NVKV_ERR_INVALID_ARG;
+    if (hidden < 64 || hidden % 64) return NVKV_ERR_UNSUPPORTED;
+    if (desc->shard_count != 1) return NVKV_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(w_k) || !aligned16(w_v)) return NVKV_ERR_ALIGNMENT;
+    return NVKV_OK;
+}
+
+nvkv::ProjLaunch project_launch(const nvkv_desc *desc, int hidden)
+{
+    nvkv::ProjLaunch p{};
+    p.T = desc->grid_h * desc->grid_w;
+    p.Lq = desc->C * p.T;
+    p.B = desc->B;
+    p.H = desc->H;
+    p.C = desc->C;
+    p.M = desc->B * p.Lq;
+    p.hidden = hidden;
+    p.R = (int)rows_per_head(desc);
+    return p;
+}
+
+}  // namespace
+
+nvkv_status nvkv_kv_project(const nvkv_desc *desc, const void *x, int hidden, const void *w_k,
+                            const void *w_v, void *k_out, void *v_out, int32_t *status,
+                            nvkv_stream stream)
+{
+    nvkv_status st = check_project(desc, x, hidden, w_k, w_v);
+    if (st != NVKV_OK) return st;
+    if (!k_out || !v_out || !status) return NVKV_ERR_INVALID_ARG;
+    if (!aligned16(k_out) || !aligned16(v_out)) return NVKV_ERR_ALIGNMENT;
+    nvkv::ProjLaunch p = project_launch(desc, hidden);
+    p.mode = 0;
+    p.k_out = k_out;
+    p.v_out = v_out;
+    p.status = status;
+    return nvkv::launch_kv_project(p, x, w_k, w_v, (cudaStream_t)stream) == cudaSuccess
+               ? NVKV_OK
+               : NVKV_ERR_CUDA;
+}
+
+nvkv_status nvfp4_kv_project_append(const nvkv_desc *desc, const nvkv_cache *cache,
+                                    nvkv_ring *ring, const void *x, int hidden, const void *w_k,
+                                    const void *w_v, void *scratch, size_t scratch_bytes,
+                                    nvkv_stream stream)
+{
+    nvkv_status st = check_project(desc, x, hidden, w_k, w_v);
+    if (st != NVKV_OK) return st;
+    if (desc->kv_dtype != NVKV_KV_NVFP4) return NVKV_ERR_STATE;
+    if ((st = check_ring(desc, ring)) != NVKV_OK) return st;
+    if (!cache || !cache->k_data || !cache->v_data || !cache->k_scales || !cache->v_scales ||
+        !cache->amax || !cache->s_g || !cache->status)
+        return NVKV_ERR_INVALID_ARG;
+    if (!aligned16(cache->k_data) || !aligned16(cache->v_data) || !aligned16(cache->k_scales) ||
+        !aligned16(cache->v_scales))
+        return NVKV_ERR_ALIGNMENT;
+    nvkv::ProjLaunch p = project_launch(desc, hidden);
+    p.status = cache->status;
+    if (!ring->scales_fixed) {
+        // first chunk: s_g comes from the whole chunk's amax, so the
+        // projection goes to bf16 first and the regular append follows
+        const size_t one = (size_t)p.M * p.H * 128 * 2;
+        if (!scratch || scratch_bytes < 2 * one) return NVKV_ERR_CAPACITY;
+        if (!aligned16(scratch)) return NVKV_ERR_ALIGNMENT;
+        {
+            int32_t slot[NVKV_MAX_BATCH * NVKV_MAX_CHUNK];
+            if (!plan_slots(desc, ring, slot)) return NVKV_ERR_CAPACITY;
+        }
+        p.mode = 0;
+        p.k_out = scratch;
+        p.v_out = static_cast<uint8_t *>(scratch) + one;
+        if (nvkv::launch_kv_project(p, x, w_k, w_v, (cudaStream_t)stream) != cudaSuccess)
+            return NVKV_ERR_CUDA;
+        return append_common(desc, cache, ring, ring, p.k_out, p.v_out, (cudaStream_t)stream,
+                             NVKV_KV_NVFP4);
+    }
+    if (!plan_slots(desc, ring, p.slot)) return NVKV_ERR_CAPACITY;
+    p.mode = 1;
+    p.k_data = cache->k_data;
+    p.v_data = cache->v_data;
+    p.k_scales = cache->k_scales;
+    p.v_scales = cache->v_scales;
+    p.s_g = cache->s_g;
+    if (nvkv::launch_kv_project(p, x, w_k, w_v, (cudaStream_t)stream) != cudaSuccess)
+        return NVKV_ERR_CUDA;
+    commit_append(desc, ring, p.slot);
+    return NVKV_OK;
+}
+
 nvkv_status nvkv_lse_merge(int n_parts, const void *const *o_parts, const float *const *lse_parts,
                            int B, int H, int Lq, int q0, int q1, void *out, float *lse_out,
                            nvkv_stream stream)

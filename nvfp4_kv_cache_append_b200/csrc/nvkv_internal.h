@@ -74,6 +74,25 @@ int attention_slots(int device);     // CTA pairs that can be resident at once
 
 cudaError_t launch_chunk_attention(const AttnLaunch &a, cudaStream_t s);
 
+// K/V projection of one chunk (x [M][hidden] times W^T, W [H*128][hidden],
+// bf16 in, f32 accumulate), its epilogue writing bf16 K/V (mode 0) or the
+// NVFP4 quantize-append into the ring (mode 1).
+struct ProjLaunch {
+    int M, hidden;                   // rows of x (B * Lq), hidden (multiple of 64)
+    int B, H, Lq, T, R, C;
+    int mode;
+    void *k_out, *v_out;             // mode 0: bf16 [B][Lq][H][128]
+    void *k_data, *v_data;           // mode 1: NVFP4 planes of the cache
+    void *k_scales, *v_scales;
+    const float *s_g;                // [2][B][H]
+    int32_t *status;
+    int n_pairs;                     // CTA pairs of the persistent grid
+    int32_t slot[NVKV_MAX_BATCH * NVKV_MAX_CHUNK];  // mode 1: [b * C + c] -> physical slot
+};
+
+cudaError_t launch_kv_project(const ProjLaunch &p, const void *x, const void *w_k, const void *w_v,
+                              cudaStream_t s);
+
 // LSE-weighted merge of the partial attentions of disjoint key sets.
 struct MergeLaunch {
     const void *o[NVKV_MAX_SHARDS];     // bf16 [B][Lq][H][128] per part
