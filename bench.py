@@ -447,6 +447,98 @@ def run_sp(args):
     dist.destroy_process_group()
 
 
+# ------------------------------------------- projection + append mode
+
+def run_project(args):
+    """--project: the K/V projection of the step's chunk (hidden = H * 128,
+    synthetic N(0, 1/hidden) weights) with the NVFP4 append fused into its
+    epilogue, against the same work as two launches (projection to bf16 K/V,
+    then the append).  Steady state (s_g fixed), 4 caches cycled."""
+    import torch
+
+    import kvsynth
+    import nvfp4_kv_cache_append_b200 as nv
+
+    ws, rank, local = _dist_env()
+    torch.cuda.set_device(local)
+    wl = kvsynth.WORKLOADS[args.workload]
+    hidden = wl.H * 128
+    g = torch.Generator().manual_seed(3)
+    xs = [torch.randn(wl.B, wl.Lq, hidden, generator=g).to(torch.bfloat16).cuda()
+          for _ in range(N_LAYERS)]
+    ws_k = [(torch.randn(wl.H * 128, hidden, generator=g) / hidden ** 0.5).to(torch.bfloat16).cuda()
+            for _ in range(N_LAYERS)]
+    ws_v = [(torch.randn(wl.H * 128, hidden, generator=g) / hidden ** 0.5).to(torch.bfloat16).cuda()
+            for _ in range(N_LAYERS)]
+    caches = [nv.KVCache(wl.B, wl.H, wl.grid_h, wl.grid_w, wl.C, wl.S, wl.W, nv.NVKV_KV_NVFP4)
+              for _ in range(N_LAYERS)]
+    k_tmp = torch.empty(wl.B, wl.Lq, wl.H, 128, dtype=torch.bfloat16, device="cuda")
+    v_tmp = torch.empty_like(k_tmp)
+    stream = torch.cuda.Stream()
+    torch.cuda.set_stream(stream)
+
+    def room(c):
+        need = wl.C - min(c.free_frames(b) for b in range(wl.B))
+        if need > 0:
+            c.evict(need)
+
+    def fused(i):
+        li = i % N_LAYERS
+        room(caches[li])
+        caches[li].project_append(xs[li], ws_k[li], ws_v[li], stream=stream)
+
+    def two(i):
+        li = i % N_LAYERS
+        c = caches[li]
+        room(c)
+        c.project(xs[li], ws_k[li], ws_v[li], k_out=k_tmp, v_out=v_tmp, stream=stream)
+        c.append(k_tmp, v_tmp, stream=stream)
+
+    for i in range(N_LAYERS * ((wl.S + wl.W) // wl.C)):      # rings full, s_g fixed
+        fused(i)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    res = {}
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    for name, fn in (("fused", fused), ("two_launch", two), ("fused_again", fused)):
+        for i in range(args.warmup):
+            fn(i)
+        torch.cuda.synchronize()
+        a, b = ev(), ev()
+        a.record(stream)
+        for i in range(args.steps):
+            fn(i)
+        b.record(stream)
+        torch.cuda.synchronize()
+        res[name] = a.elapsed_time(b) / args.steps
+    clk = clocks.stop()
+    for c in caches:
+        assert c.device_status() == 0, "device-side pipeline error"
+    fused_ms = min(res["fused"], res["fused_again"])
+    flop = 2.0 * wl.B * wl.Lq * hidden * 2 * wl.H * 128
+    peaks = _peaks()
+    tflops = flop / (fused_ms / 1e3) / 1e12
+    line = {
+        "metric": "fused K/V projection + NVFP4 append, ms per step", "value": fused_ms,
+        "unit": "ms", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": fused_ms, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 MMA, f32 accumulate, e2m1/e4m3 out",
+        "data": "synthetic (seeded N(0,1) hidden states, N(0, 1/hidden) weights)",
+        "config": {"workload": bench_config(wl, "nvfp4", 1)["workload"], "hidden": hidden,
+                   "gemm": f"M={wl.B * wl.Lq} N={2 * wl.H * 128} K={hidden}",
+                   "l2": "4 input/weight sets and caches cycled"},
+        "two_launch_ms": res["two_launch"],
+        "fused_gain": res["two_launch"] / fused_ms,
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"], "traffic": None,
+                     "kernel": "k_kv_project", "peak_source": peaks["source"] + " bf16"},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------ oracle arm
 
 class OracleSample:
@@ -568,6 +660,8 @@ def main():
     ap.add_argument("--kv", default="nvfp4", choices=["nvfp4", "bf16"])
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--project", action="store_true",
+                    help="time the fused K/V projection + append against two launches")
     ap.add_argument("--sp", action="store_true",
                     help="sequence-parallel KV split over the ranks instead of replicas")
     args = ap.parse_args()
@@ -577,6 +671,8 @@ def main():
         run_reference(args)
     elif args.sp:
         run_sp(args)
+    elif args.project:
+        run_project(args)
     else:
         run_ours(args)
 

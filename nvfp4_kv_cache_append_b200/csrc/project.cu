@@ -10,14 +10,17 @@
 // generation", section "NVFP4, sequence parallel and the async decode path";
 // the bf16 K/V never reaches HBM).
 //
-// Structure: a cluster of two CTAs (one per SM) computes a 256 x 128 output
-// tile: 256 token rows (128 per CTA) by the 128 channels of one head of K or
-// V.  Every MMA is a pair MMA (cta_group::2, M = 256, N = 128, both operands
-// in shared memory, 128-byte swizzle), issued by the even CTA; each CTA
-// stages its own 128 rows of x and its 64-row half of the head's weights per
-// 64-element step of hidden, by TMA, in a 6-stage ring.  The accumulator is
-// double buffered in TMEM so that the epilogue of one tile overlaps the MMAs
-// of the next.  Warps:
+// Structure: a cluster of two CTAs (one per SM) computes a 256 x 256 output
+// tile: 256 token rows (128 per CTA) by the 128 channels of each of two
+// heads (of K, of V, or one of each).  Every MMA is a pair MMA (cta_group::2,
+// M = 256, N = 256, both operands in shared memory, 128-byte swizzle), issued
+// by the even CTA; per 64-element step of hidden each CTA stages, by TMA, its
+// own 128 rows of x and the 128 weight rows of its head of the pair (B is
+// split along N between the two CTAs), in a 6-stage ring.  Against 256 x 128
+// tiles this cuts the operand traffic from L2 per FLOP by a third, which is
+// what bounds the kernel.  The accumulator (256 columns) is double buffered
+// in TMEM so that the epilogue of one tile overlaps the MMAs of the next.
+// Warps:
 //   warp 0       producer (TMA) in both CTAs
 //   warp 1       TMEM allocation; MMA issuer (even CTA) or relay of the
 //                stage-full events (odd CTA)
@@ -40,7 +43,7 @@ constexpr int PM = 128;                            // rows per CTA
 constexpr int PK = 64;                             // hidden elements per stage
 constexpr int NST = 6;                             // stages
 constexpr uint32_t A_BYTES = PM * PK * 2;          // 16 KB
-constexpr uint32_t B_BYTES = 64 * PK * 2;          // 8 KB: 64 of the head's 128 channels
+constexpr uint32_t B_BYTES = 128 * PK * 2;         // 16 KB: one head's 128 channels
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int PTHREADS = 256;
 constexpr uint64_t PWAIT_NS = 2000000000ull;       // 2 s per wait
@@ -102,9 +105,9 @@ __device__ void producer(PCtx &c, const CUtensorMap *tx, const CUtensorMap *twk,
     int it = 0;
     bool ok = true;
     for (int t = c.pair; ok && t < c.n_tiles; t += p.n_pairs) {
-        const int mt = t / (2 * p.H), nt = t - mt * (2 * p.H);
-        const CUtensorMap *tw = nt < p.H ? twk : twv;
-        const int wrow = (nt < p.H ? nt : nt - p.H) * 128 + 64 * (int)c.rank;
+        const int mt = t / p.H, hh = 2 * (t - mt * p.H) + (int)c.rank;   // this CTA's head
+        const CUtensorMap *tw = hh < p.H ? twk : twv;
+        const int wrow = (hh < p.H ? hh : hh - p.H) * 128;
         const int xrow = mt * 2 * PM + PM * (int)c.rank;
         for (int ks = 0; ks < c.nk; ++ks, ++it) {
             const int s = it % NST;
@@ -126,7 +129,7 @@ __device__ void mma_issuer(PCtx &c)
 {
     const ProjLaunch &p = *c.p;
     const uint32_t tmem = c.ctl->tmem_base;
-    constexpr uint32_t idesc = ptx::idesc_f16(1 /* bf16 */, 2 * PM, 128, 0);
+    constexpr uint32_t idesc = ptx::idesc_f16(1 /* bf16 */, 2 * PM, 256, 0);
     const uint16_t both = 0x3;
     int it = 0, j = 0;
     bool ok = true;
@@ -142,7 +145,7 @@ __device__ void mma_issuer(PCtx &c)
             const uint32_t a0 = ptx::smem_u32(c.stages + s * STAGE_BYTES), b0 = a0 + A_BYTES;
 #pragma unroll
             for (int kk = 0; kk < PK / 16; ++kk)
-                ptx::mma2_f16_ss(tmem + b * 128, ptx::smem_desc_sw128(a0 + kk * 32, 16, 1024),
+                ptx::mma2_f16_ss(tmem + b * 256, ptx::smem_desc_sw128(a0 + kk * 32, 16, 1024),
                                  ptx::smem_desc_sw128(b0 + kk * 32, 16, 1024), idesc,
                                  (ks | kk) ? 1u : 0u);
             ptx::mma2_commit_mc(&c.ctl->bar[P_EMPTY + s], both);
@@ -194,44 +197,53 @@ __device__ void epilogue(PCtx &c)
         const int b = j & 1;
         if (!pwait_warp(c, P_AFULL + b, (j >> 1) & 1)) return;
         ptx::tc_fence_after();
-        const int mt = t / (2 * p.H), nt = t - mt * (2 * p.H);
-        const int kv = nt < p.H ? 0 : 1, h = nt - kv * p.H;
+        const int mt = t / p.H;
         const int row = mt * 2 * PM + PM * (int)c.rank + r;
         const bool valid = row < p.M;
         const int bi = valid ? row / p.Lq : 0, l = valid ? row - bi * p.Lq : 0;
-        size_t drow = 0;
-        float sg = 1.0f;
+        int frame = 0, tok = 0;
         if (p.mode == 1) {
-            const int frame = l / p.T, tok = l - frame * p.T;
-            drow = (size_t)(bi * p.H + h) * p.R + (size_t)p.slot[bi * p.C + frame] * p.T + tok;
-            sg = p.s_g[(kv * p.B + bi) * p.H + h];
+            frame = l / p.T;
+            tok = l - frame * p.T;
         }
 #pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-            uint32_t v[32];
-            ptx::tmem_ld32(tbase + b * 128 + q * 32, v);
-            ptx::tmem_wait_ld();
-            uint32_t w[16];
+        for (int half = 0; half < 2; ++half) {
+            const int hh = 2 * (t - mt * p.H) + half;          // head of columns [128 half, +128)
+            const int kv = hh < p.H ? 0 : 1, h = hh - kv * p.H;
+            size_t drow = 0;
+            float sg = 1.0f;
+            if (p.mode == 1) {
+                drow = (size_t)(bi * p.H + h) * p.R + (size_t)p.slot[bi * p.C + frame] * p.T + tok;
+                sg = p.s_g[(kv * p.B + bi) * p.H + h];
+            }
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                uint32_t v[32];
+                ptx::tmem_ld32(tbase + b * 256 + half * 128 + q * 32, v);
+                ptx::tmem_wait_ld();
+                uint32_t w[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                w[i] = bf16x2_bits(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-            if (!valid) continue;
-            if (p.mode == 0) {
-                uint4 *dst = reinterpret_cast<uint4 *>(kv ? p.v_out : p.k_out) +
-                             (((size_t)bi * p.Lq + l) * p.H + h) * 16 + q * 4;
+                for (int i = 0; i < 16; ++i)
+                    w[i] = bf16x2_bits(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                if (!valid) continue;
+                if (p.mode == 0) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(kv ? p.v_out : p.k_out) +
+                                 (((size_t)bi * p.Lq + l) * p.H + h) * 16 + q * 4;
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-            } else {
-                uint2 c0, c1;
-                const uint32_t s0 = q4::quantize_block(make_uint4(w[0], w[1], w[2], w[3]),
-                                                       make_uint4(w[4], w[5], w[6], w[7]), sg, c0);
-                const uint32_t s1 = q4::quantize_block(make_uint4(w[8], w[9], w[10], w[11]),
-                                                       make_uint4(w[12], w[13], w[14], w[15]), sg, c1);
-                *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(kv ? p.v_data : p.k_data) +
-                                           drow * 64 + q * 16) = make_uint4(c0.x, c0.y, c1.x, c1.y);
-                *reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(kv ? p.v_scales : p.k_scales) +
-                                              drow * 8 + q * 2) = (uint16_t)(s0 | (s1 << 8));
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                } else {
+                    uint2 c0, c1;
+                    const uint32_t s0 = q4::quantize_block(make_uint4(w[0], w[1], w[2], w[3]),
+                                                           make_uint4(w[4], w[5], w[6], w[7]), sg, c0);
+                    const uint32_t s1 = q4::quantize_block(make_uint4(w[8], w[9], w[10], w[11]),
+                                                           make_uint4(w[12], w[13], w[14], w[15]), sg,
+                                                           c1);
+                    *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(kv ? p.v_data : p.k_data) +
+                                               drow * 64 + q * 16) = make_uint4(c0.x, c0.y, c1.x, c1.y);
+                    *reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(kv ? p.v_scales : p.k_scales) +
+                                                  drow * 8 + q * 2) = (uint16_t)(s0 | (s1 << 8));
+                }
             }
         }
         ptx::tc_fence_before();
@@ -253,7 +265,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
     c.rank = ptx::cluster_ctarank();
     c.pair = blockIdx.x >> 1;
     c.nk = p.hidden / PK;
-    c.n_tiles = (p.M + 2 * PM - 1) / (2 * PM) * 2 * p.H;
+    c.n_tiles = (p.M + 2 * PM - 1) / (2 * PM) * p.H;
     c.lead_bar = ptx::mapa(ptx::smem_u32(&c.ctl->bar[0]), 0);
     c.peer_abort = ptx::mapa(ptx::smem_u32(&c.ctl->abort), c.rank ^ 1u);
     const int warp = threadIdx.x >> 5;
@@ -268,7 +280,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
         ptx::fence_mbar_init();
     }
     if (warp == 1) {
-        ptx::tmem_alloc2(&c.ctl->tmem_base, 256);
+        ptx::tmem_alloc2(&c.ctl->tmem_base, 512);
         ptx::tmem_relinquish2();
     }
     ptx::tc_fence_before();
@@ -298,7 +310,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
     ptx::cluster_sync();          // no CTA leaves while its peer may touch its memory
     if (warp == 1) {
         ptx::tc_fence_after();
-        ptx::tmem_dealloc2(c.ctl->tmem_base, 256);
+        ptx::tmem_dealloc2(c.ctl->tmem_base, 512);
     }
 }
 
@@ -344,14 +356,14 @@ cudaError_t launch_kv_project(const ProjLaunch &p_in, const void *x, const void 
     ProjLaunch p = p_in;
     CUtensorMap tx, twk, twv;
     if (!make_map(&tx, x, (uint64_t)p.M, (uint64_t)p.hidden, PM) ||
-        !make_map(&twk, w_k, (uint64_t)p.H * 128, (uint64_t)p.hidden, 64) ||
-        !make_map(&twv, w_v, (uint64_t)p.H * 128, (uint64_t)p.hidden, 64))
+        !make_map(&twk, w_k, (uint64_t)p.H * 128, (uint64_t)p.hidden, 128) ||
+        !make_map(&twv, w_v, (uint64_t)p.H * 128, (uint64_t)p.hidden, 128))
         return cudaErrorInvalidValue;
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    const int n_tiles = (p.M + 2 * PM - 1) / (2 * PM) * 2 * p.H;
+    const int n_tiles = (p.M + 2 * PM - 1) / (2 * PM) * p.H;
     p.n_pairs = sms / 2 < n_tiles ? sms / 2 : n_tiles;
     if (p.n_pairs < 1) return cudaErrorInvalidConfiguration;
     const int bytes = 1024 + NST * STAGE_BYTES + (int)sizeof(PCtl);
