@@ -75,7 +75,7 @@ class NvkvError(RuntimeError):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"libnvkv.so not built at {LIB_PATH}; run "
-                          "`python -m nvfp4_kv_cache_append_b200.build` (needs nvcc)")
+                          "`python nvfp4_kv_cache_append_b200/build.py` (needs nvcc)")
     L = ctypes.CDLL(LIB_PATH)
     D, C, R = ctypes.POINTER(nvkv_desc), ctypes.POINTER(nvkv_cache), ctypes.POINTER(nvkv_ring)
     vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
