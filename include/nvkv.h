@@ -358,6 +358,18 @@ NVKV_API nvkv_status nvkv_lse_merge(int n_parts, const void *const *o_parts,
                                     const float *const *lse_parts, int B, int H, int Lq, int q0,
                                     int q1, void *out, float *lse_out, nvkv_stream stream);
 
+/* Test hook of the failure path (no counterpart in the paper).  With fault =
+ * NVKV_FAULT_SKIP_FIRST_STAGE the next chunk_attention_* call on this thread
+ * runs with its staging producer never filling the first stage, so the waits
+ * on it run out after their bound (2 s): the kernel writes NVKV_ERR_TIMEOUT
+ * to cache->status, unwinds (waiting for its own copies and MMAs) and
+ * returns; nothing traps or hangs.  After a timeout the caller clears the
+ * status word and zero-fills the workspace again before reusing them; the
+ * output of that call is undefined.  NVKV_FAULT_NONE cancels a pending
+ * fault. */
+enum { NVKV_FAULT_NONE = 0, NVKV_FAULT_SKIP_FIRST_STAGE = 1 };
+NVKV_API nvkv_status nvkv_debug_inject_fault(int fault);
+
 /* Diagnostics: the device conversions the append kernel uses, one value per
  * element.  y, t: device f32 [n]; codes: device u8 [n].
  * nvkv_encode_e2m1: E2M1_RNE_sat(y) with negative zero stored as 0.

@@ -84,6 +84,7 @@ def _load():
         "nvkv_desc_init": (i32, [D, i32, i32, i32, i32, i32, i32, i32, i32]),
         "nvkv_desc_set_shard": (i32, [D, i32, i32]),
         "nvkv_kv_project": (i32, [D, vp, i32, vp, vp, vp, vp, vp, vp]),
+        "nvkv_debug_inject_fault": (i32, [i32]),
         "nvfp4_kv_project_append": (i32, [D, C, R, vp, i32, vp, vp, vp, sz, vp]),
         "nvkv_lse_merge": (i32, [i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, i32,
                                  i32, vp, vp, vp]),
@@ -149,6 +150,14 @@ def nvkv_lse_merge(o_ptrs, lse_ptrs, B, H, Lq, q0, q1, out_ptr, lse_out_ptr=None
     la = (ctypes.c_void_p * max(n, 1))(*lse_ptrs)
     _check(lib.nvkv_lse_merge(n, oa, la, B, H, Lq, q0, q1, out_ptr, lse_out_ptr, stream),
            "nvkv_lse_merge")
+
+
+NVKV_FAULT_NONE = 0
+NVKV_FAULT_SKIP_FIRST_STAGE = 1
+
+
+def nvkv_debug_inject_fault(fault: int) -> None:
+    _check(lib.nvkv_debug_inject_fault(fault), "nvkv_debug_inject_fault")
 
 
 def nvkv_kv_project(desc, x_ptr, hidden, wk_ptr, wv_ptr, k_out_ptr, v_out_ptr, status_ptr,

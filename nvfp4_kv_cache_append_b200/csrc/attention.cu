@@ -682,17 +682,23 @@ __device__ __forceinline__ void copy_runs(const AttnLaunch &a, int b, size_t hea
     }
 }
 
+// FAULT: the failure-path test variant (nvkv_debug_inject_fault): the first
+// stage is never filled, so the waits on it run out
+template <bool FAULT>
 __device__ void producer_role(Ctx &c)
 {
     const AttnLaunch &a = *c.a;
     int g = 0;
-    for (int si = 0; si < c.ctl->n_seg; ++si) {
+    bool ok = true;
+    for (int si = 0; ok && si < c.ctl->n_seg; ++si) {
         const Segment sg = c.ctl->seg[si];
         const int n_keys = a.n_vis[sg.b] * a.Tk;
         const size_t head_row0 = (size_t)(sg.b * a.H + sg.h) * a.R;
         for (int tile = sg.t0; tile < sg.t1; ++tile, ++g) {
             const int s = g % NSTAGE;
-            if (g >= NSTAGE && !wait(c, B_STG_EMPTY + s, ((g - NSTAGE) / NSTAGE) & 1)) return;
+            if (g >= NSTAGE && !(ok = wait(c, B_STG_EMPTY + s, ((g - NSTAGE) / NSTAGE) & 1)))
+                break;
+            if (FAULT && g == 0) continue;
             uint8_t *stg = c.smem + OFF_STG + s * STG_BYTES;
             uint64_t *full = &c.ctl->bar[B_STG_FULL + s];
             const int kk0 = min(n_keys, tile * BN + 64 * (int)c.rank);
@@ -707,6 +713,14 @@ __device__ void producer_role(Ctx &c)
                       static_cast<const uint8_t *>(a.v_data),
                       static_cast<const uint8_t *>(a.v_scales), full);
         }
+    }
+    // no CTA leaves with copies into its shared memory in flight (after an
+    // abort, stages nobody consumed may still be landing)
+    const int never = 0;
+    for (int i = g - 1; i >= 0 && i >= g - NSTAGE; --i) {
+        if (FAULT && i == 0) continue;
+        ptx::mbar_wait(&c.ctl->bar[B_STG_FULL + i % NSTAGE], (i / NSTAGE) & 1, &never,
+                       WAIT_LIMIT_NS);
     }
 }
 
@@ -995,9 +1009,10 @@ __device__ void softmax_role(Ctx &c)
 
 // ------------------------------------------------------------ kernel
 
-// SHARD: the cache is a shard whose first token is not token 0 of the frame;
-// a separate instantiation keeps the whole-cache kernel's code as it was
-template <bool FP4, bool SHARD>
+// VAR 0: a whole cache; 1 (SHARD): a shard whose first token is not token 0
+// of the frame; 2: the failure-path test.  Separate instantiations keep the
+// whole-cache kernel's code free of both.
+template <bool FP4, int VAR>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     k_chunk_attn(const __grid_constant__ AttnLaunch a)
 {
@@ -1047,11 +1062,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     if (warp < 4) {
         softmax_role<FP4>(c);
     } else if (warp < 8) {
-        k_converter_role<FP4, SHARD>(c);
+        k_converter_role<FP4, VAR == 1>(c);
     } else if (warp < 12) {
-        v_converter_role<FP4, SHARD>(c);
+        v_converter_role<FP4, VAR == 1>(c);
     } else if (warp == 12) {
-        if (FP4 && (threadIdx.x & 31) == 0) producer_role(c);
+        if (FP4 && (threadIdx.x & 31) == 0) producer_role<VAR == 2>(c);
     } else if (warp == 13) {
         if ((threadIdx.x & 31) == 0) {
             if (c.rank == 0) mma_role(c);
@@ -1076,18 +1091,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     }
 }
 
-template <bool FP4, bool SHARD>
+template <bool FP4, int VAR>
 cudaError_t launch(const AttnLaunch &a, cudaStream_t s)
 {
     const uint32_t tab =
         (uint32_t)(a.n_fpos * PAIRS_F + a.grid_h * PAIRS_H + a.grid_w * PAIRS_W) * 8;
     const uint32_t bytes = 1024 + OFF_TAB + ((tab + 63) & ~63u) + sizeof(SharedCtl);
     if (bytes > 232448) return cudaErrorInvalidConfiguration;
-    cudaError_t e = cudaFuncSetAttribute(k_chunk_attn<FP4, SHARD>,
+    cudaError_t e = cudaFuncSetAttribute(k_chunk_attn<FP4, VAR>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
     const dim3 grid(2 * a.n_slots, 1, 1);
-    k_chunk_attn<FP4, SHARD><<<grid, NTHREADS, bytes, s>>>(a);
+    k_chunk_attn<FP4, VAR><<<grid, NTHREADS, bytes, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -1109,9 +1124,10 @@ int attention_slots(int device)
 
 cudaError_t launch_chunk_attention(const AttnLaunch &a, cudaStream_t s)
 {
-    if (a.tok_off)
-        return a.kv_dtype == NVKV_KV_NVFP4 ? launch<true, true>(a, s) : launch<false, true>(a, s);
-    return a.kv_dtype == NVKV_KV_NVFP4 ? launch<true, false>(a, s) : launch<false, false>(a, s);
+    const bool fp4 = a.kv_dtype == NVKV_KV_NVFP4;
+    if (fp4 && a.fault == NVKV_FAULT_SKIP_FIRST_STAGE && !a.tok_off) return launch<true, 2>(a, s);
+    if (a.tok_off) return fp4 ? launch<true, 1>(a, s) : launch<false, 1>(a, s);
+    return fp4 ? launch<true, 0>(a, s) : launch<false, 0>(a, s);
 }
 
 }  // namespace nvkv

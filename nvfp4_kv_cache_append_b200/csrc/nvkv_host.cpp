@@ -189,6 +189,8 @@ nvkv_status append_common(const nvkv_desc *desc, const nvkv_cache *cache, const 
 // tiles per slot.  Each slot holds at most kMaxSegments work segments, so
 // very small items raise the slot count (extra pairs run as later waves).
 constexpr int kTileKeys = 128;
+// one-shot test hook (nvkv_debug_inject_fault), consumed by the next attention call
+thread_local int t_fault = NVKV_FAULT_NONE;
 constexpr int kMaxSegments = 94;     // the kernel holds 96; two spare
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -287,6 +289,8 @@ nvkv_status attention_common(const nvkv_desc *desc, const nvkv_cache *cache,
     if (!ws || ws_bytes < nvkv::attention_workspace_bytes(a.n_slots)) return NVKV_ERR_CAPACITY;
     if (reinterpret_cast<uintptr_t>(ws) & 15u) return NVKV_ERR_ALIGNMENT;
     a.workspace = ws;
+    a.fault = t_fault;
+    t_fault = NVKV_FAULT_NONE;
     if (nvkv::launch_chunk_attention(a, stream) != cudaSuccess) return NVKV_ERR_CUDA;
     return NVKV_OK;
 }
@@ -626,6 +630,14 @@ nvkv_status nvkv_lse_merge(int n_parts, const void *const *o_parts, const float 
     m.out = out;
     m.lse_out = lse_out;
     return nvkv::launch_lse_merge(m, (cudaStream_t)stream) == cudaSuccess ? NVKV_OK : NVKV_ERR_CUDA;
+}
+
+nvkv_status nvkv_debug_inject_fault(int fault)
+{
+    if (fault != NVKV_FAULT_NONE && fault != NVKV_FAULT_SKIP_FIRST_STAGE)
+        return NVKV_ERR_INVALID_ARG;
+    t_fault = fault;
+    return NVKV_OK;
 }
 
 nvkv_status nvkv_encode_e2m1(const float *y, uint8_t *codes, size_t n, nvkv_stream stream)

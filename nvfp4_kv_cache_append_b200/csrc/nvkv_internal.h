@@ -65,6 +65,7 @@ struct AttnLaunch {
     void *workspace;                 // split-item partials + counters (zero on first use)
     int n_slots;                     // CTA pairs of the persistent schedule
     int n_pairs;                     // 256-row query tile pairs per (b, h)
+    int fault;                       // NVKV_FAULT_* test hook, 0 in normal use
 };
 
 // Workspace of the chunk attention for a schedule of n_slots CTA pairs:

@@ -224,3 +224,8 @@ def test_status_strings():
     for code, name in L.STATUS.items():
         assert nv.nvkv_status_string(code)
     assert "unknown" in nv.nvkv_status_string(99)
+
+
+def test_fault_hook_validation():
+    assert _status(L.nvkv_debug_inject_fault, 9) == "NVKV_ERR_INVALID_ARG"
+    assert _status(L.nvkv_debug_inject_fault, L.NVKV_FAULT_NONE) == "NVKV_OK"
