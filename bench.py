@@ -39,16 +39,17 @@ def _peaks():
             "source": "fallback"}
 
 
-def _ncu_traffic(kernel: str):
-    """DRAM bytes per launch from the committed ncu capture, or None when the
-    kernel's sources changed since the counters were taken."""
+def _ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu capture of this kernel on
+    this workload, or None when there is none or the kernel's sources changed
+    since the counters were taken."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f).get(kernel)
-    if not d:
+    if not d or not d["workload"].startswith(workload + " "):
         return None
     h = hashlib.sha256()
     for src in d["sources"]:
@@ -340,7 +341,7 @@ def run_ours(args):
         "append_ms": app_avg,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak,
                      "unit": "TFLOP/s", "frac": attn_tflops / peak,
-                     "traffic": _ncu_traffic("k_chunk_attn<1, 0>") if fp4 else None,
+                     "traffic": _ncu_traffic("k_chunk_attn<1, 0>", wl.name) if fp4 else None,
                      "kernel": "k_chunk_attn", "peak_source": peaks["source"] + " bf16 (f16 same nominal rate)"},
         "append_roofline": {"bound": "hbm", "achieved": append_gbs, "peak": peaks["hbm_gbs"],
                             "unit": "GB/s", "frac": append_gbs / peaks["hbm_gbs"]},
