@@ -142,3 +142,32 @@ def test_projection_rejects_bad_arguments():
     with pytest.raises(L.NvkvError):          # shards: not supported
         s.project(x, w, w)
     assert c.ring.steps == 0
+
+
+def test_projection_odd_heads_two_streams():
+    # H = 3: a 256-channel tile holds K head 2 and V head 0; B = 2: one row
+    # tile spans both streams; T = 20 tokens, hidden = 64 (one stage per tile)
+    import nvfp4_kv_cache_append_b200 as nv
+    wl = kvsynth.Workload("oddh", B=2, H=3, D=128, grid_h=4, grid_w=5, C=2, S=1, W=3, steps=4)
+    fused = LibStream(wl, nv.NVKV_KV_NVFP4)
+    ora = OracleStream(wl, seed=0, keep_inputs=False)
+    for step in range(1, wl.steps + 1):
+        x, wk, wv = _exact_inputs(wl, 64, step)
+        kref, vref = _oracle_kv(x, wk, wl), _oracle_kv(x, wv, wl)
+        q = kvsynth.chunk_qkv(wl, step, 0, which="q")["q"]
+        new = ora.step(k=kref, v=vref, q=q)
+        k, v = fused.cache.project(x.cuda(), wk.cuda(), wv.cuda())
+        _make_room(fused.cache)
+        fused.cache.project_append(x.cuda(), wk.cuda(), wv.cuda())
+        torch.cuda.synchronize()
+        assert fused.cache.device_status() == 0
+        assert torch.equal(k.cpu(), kref) and torch.equal(v.cpu(), vref)
+        for b in range(wl.B):
+            for fid in new[b]:
+                rows = fused.frame_rows(b, fid)
+                e = ora.frame(b, fid)
+                for w in ("k", "v"):
+                    assert np.array_equal(fused.cache.codes(w)[b, :, rows].cpu().numpy(),
+                                          e[w + "_codes"]), (step, b, fid, w)
+                    assert np.array_equal(fused.cache.scales(w)[b, :, rows].cpu().numpy(),
+                                          e[w + "_scales"]), (step, b, fid, w)
