@@ -448,6 +448,69 @@ def run_sp(args):
     dist.destroy_process_group()
 
 
+# ------------------------------------------ one-GPU shard emulation mode
+
+def run_sp_emulate(args):
+    """--sp-emulate: the per-rank kernel times of the sequence-parallel split
+    for N = 1, 2, 3, 4, 6 shards, all run on this one GPU: one shard's
+    attention over its 1/N of every frame's tokens, and the merge of one
+    rank's query slice from the N shards' partial results (local here; over
+    NVLink on N GPUs).  L2 is flushed (256 MB written) before every timed
+    launch.  Prints one JSON line."""
+    import torch
+
+    import kvsynth
+    import nvfp4_kv_cache_append_b200 as nv
+
+    torch.cuda.set_device(0)
+    wl = kvsynth.WORKLOADS[args.workload]
+    x = {k: v.cuda() for k, v in kvsynth.chunk_qkv(wl, 1000, 0).items()}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def timed(fn, n):
+        ms = []
+        for i in range(n + 3):
+            flush.fill_(i & 0xFF)
+            a, b = ev(), ev()
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                ms.append(a.elapsed_time(b))
+        return statistics.median(ms)
+
+    rows = []
+    for n in (1, 2, 3, 4, 6):
+        if wl.T % n or (wl.T // n) % 2:
+            continue
+        shards = [nv.KVCache(wl.B, wl.H, wl.grid_h, wl.grid_w, wl.C, wl.S, wl.W, nv.NVKV_KV_NVFP4,
+                             shard_rank=r, shard_count=n) for r in range(n)]
+        outs = [torch.empty_like(x["q"]) for _ in range(n)]
+        lses = [torch.empty(wl.B, wl.H, wl.Lq, device="cuda") for _ in range(n)]
+        for _ in range((wl.S + wl.W) // wl.C):
+            for r, c in enumerate(shards):
+                c.step(x["q"], x["k"], x["v"], out=outs[r], lse=lses[r])
+        torch.cuda.synchronize()
+        c = shards[-1]
+        att = timed(lambda: c.attention(x["q"], out=outs[-1], lse=lses[-1]), args.steps)
+        q1 = wl.Lq // n
+        mo = torch.empty(wl.B, q1, wl.H, 128, dtype=torch.bfloat16, device="cuda")
+        mrg = timed(lambda: nv.lse_merge(outs, lses, 0, q1, out=mo), args.steps)
+        assert all(s_.device_status() == 0 for s_ in shards)
+        rows.append({"shards": n, "shard_attention_ms": att, "merge_ms": mrg,
+                     "cache_bytes_per_rank": shards[0].footprint_bytes()})
+        del shards, outs, lses
+    base = rows[0]["shard_attention_ms"] + rows[0]["merge_ms"]
+    for r in rows:
+        r["attention_plus_merge_speedup"] = base / (r["shard_attention_ms"] + r["merge_ms"])
+    print(json.dumps({"metric": "sequence-parallel split, per-rank kernel times emulated on one GPU",
+                      "workload": bench_config(wl, "nvfp4", 1)["workload"],
+                      "l2": "256 MB written before every timed launch", "steps": args.steps,
+                      "rows": rows}), flush=True)
+
+
 # ------------------------------------------- projection + append mode
 
 def run_project(args):
@@ -661,6 +724,8 @@ def main():
     ap.add_argument("--kv", default="nvfp4", choices=["nvfp4", "bf16"])
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sp-emulate", action="store_true",
+                    help="per-rank kernel times of the sequence-parallel split, emulated on one GPU")
     ap.add_argument("--project", action="store_true",
                     help="time the fused K/V projection + append against two launches")
     ap.add_argument("--sp", action="store_true",
@@ -674,6 +739,8 @@ def main():
         run_sp(args)
     elif args.project:
         run_project(args)
+    elif args.sp_emulate:
+        run_sp_emulate(args)
     else:
         run_ours(args)
 
