@@ -72,7 +72,23 @@ struct PCtx {
     uint32_t lead_bar;             // shared::cluster address of the even CTA's bar[0]
     uint32_t peer_abort;
     int n_tiles, nk, pair;
+    int n_full, n_items;           // tiles in whole waves; work items (see item_of)
 };
+
+// Work item v of the persistent schedule.  Tiles are 256 x 256 (two heads);
+// when the tiles left after the last whole wave fit twice into one wave,
+// each of them runs as two 256 x 128 halves (one head each, N = 128 MMAs) on
+// two pairs, which halves that wave's length.  half = -1: the whole tile.
+struct Item {
+    int t, half;
+};
+
+__device__ __forceinline__ Item item_of(const PCtx &c, int v)
+{
+    if (v < c.n_full) return {v, -1};
+    const int h = v - c.n_full;
+    return {c.n_full + (h >> 1), h & 1};
+}
 
 __device__ __forceinline__ void pset_abort(PCtx &c)
 {
@@ -104,10 +120,14 @@ __device__ void producer(PCtx &c, const CUtensorMap *tx, const CUtensorMap *twk,
     ptx::prefetch_tensormap(twv);
     int it = 0;
     bool ok = true;
-    for (int t = c.pair; ok && t < c.n_tiles; t += p.n_pairs) {
-        const int mt = t / p.H, hh = 2 * (t - mt * p.H) + (int)c.rank;   // this CTA's head
+    for (int v = c.pair; ok && v < c.n_items; v += p.n_pairs) {
+        const Item w = item_of(c, v);
+        const int mt = w.t / p.H, tt = w.t - mt * p.H;
+        // whole tile: this CTA's head of the pair; half tile: this CTA's 64
+        // rows of the one head (the box's other 64 rows go unused)
+        const int hh = 2 * tt + (w.half < 0 ? (int)c.rank : w.half);
         const CUtensorMap *tw = hh < p.H ? twk : twv;
-        const int wrow = (hh < p.H ? hh : hh - p.H) * 128;
+        const int wrow = (hh < p.H ? hh : hh - p.H) * 128 + (w.half < 0 ? 0 : 64 * (int)c.rank);
         const int xrow = mt * 2 * PM + PM * (int)c.rank;
         for (int ks = 0; ks < c.nk; ++ks, ++it) {
             const int s = it % NST;
@@ -129,11 +149,13 @@ __device__ void mma_issuer(PCtx &c)
 {
     const ProjLaunch &p = *c.p;
     const uint32_t tmem = c.ctl->tmem_base;
-    constexpr uint32_t idesc = ptx::idesc_f16(1 /* bf16 */, 2 * PM, 256, 0);
+    constexpr uint32_t idesc256 = ptx::idesc_f16(1 /* bf16 */, 2 * PM, 256, 0);
+    constexpr uint32_t idesc128 = ptx::idesc_f16(1 /* bf16 */, 2 * PM, 128, 0);
     const uint16_t both = 0x3;
     int it = 0, j = 0;
     bool ok = true;
-    for (int t = c.pair; ok && t < c.n_tiles; t += p.n_pairs, ++j) {
+    for (int v = c.pair; ok && v < c.n_items; v += p.n_pairs, ++j) {
+        const uint32_t idesc = item_of(c, v).half < 0 ? idesc256 : idesc128;
         const int b = j & 1;
         if (j >= 2 && !(ok = pwait(c, P_AEMPTY + b, ((j - 2) >> 1) & 1))) break;
         ptx::tc_fence_after();
@@ -161,7 +183,7 @@ __device__ void relay_full(PCtx &c)
 {
     const ProjLaunch &p = *c.p;
     int it = 0;
-    for (int t = c.pair; t < c.n_tiles; t += p.n_pairs)
+    for (int v = c.pair; v < c.n_items; v += p.n_pairs)
         for (int ks = 0; ks < c.nk; ++ks, ++it) {
             const int s = it % NST;
             if (!pwait(c, P_FULL + s, (it / NST) & 1)) return;
@@ -174,7 +196,7 @@ __device__ void relay_aempty(PCtx &c)
 {
     const ProjLaunch &p = *c.p;
     int j = 0;
-    for (int t = c.pair; t < c.n_tiles; t += p.n_pairs, ++j) {
+    for (int v = c.pair; v < c.n_items; v += p.n_pairs, ++j) {
         const int b = j & 1;
         if (!pwait(c, P_AEMPTY + b, (j >> 1) & 1)) return;
         ptx::mbar_arrive_remote(c.lead_bar + (P_AEMPTY + b) * 8);
@@ -193,11 +215,12 @@ __device__ void epilogue(PCtx &c)
     const int r = threadIdx.x - 128;                   // TMEM lane = row of the CTA's half
     const uint32_t tbase = c.ctl->tmem_base + ((uint32_t)(r & ~31) << 16);
     int j = 0;
-    for (int t = c.pair; t < c.n_tiles; t += p.n_pairs, ++j) {
+    for (int v = c.pair; v < c.n_items; v += p.n_pairs, ++j) {
         const int b = j & 1;
         if (!pwait_warp(c, P_AFULL + b, (j >> 1) & 1)) return;
         ptx::tc_fence_after();
-        const int mt = t / p.H;
+        const Item wi = item_of(c, v);
+        const int t = wi.t, mt = t / p.H;
         const int row = mt * 2 * PM + PM * (int)c.rank + r;
         const bool valid = row < p.M;
         const int bi = valid ? row / p.Lq : 0, l = valid ? row - bi * p.Lq : 0;
@@ -206,9 +229,13 @@ __device__ void epilogue(PCtx &c)
             frame = l / p.T;
             tok = l - frame * p.T;
         }
+        const int h0 = wi.half < 0 ? 0 : wi.half, h1 = wi.half < 0 ? 2 : wi.half + 1;
 #pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-            const int hh = 2 * (t - mt * p.H) + half;          // head of columns [128 half, +128)
+        for (int hs = h0; hs < h1; ++hs) {
+            // head of accumulator columns [128 col, +128): the tile's two
+            // heads in turn, or the half tile's one head in columns 0-127
+            const int hh = 2 * (t - mt * p.H) + hs;
+            const int col = wi.half < 0 ? hs : 0;
             const int kv = hh < p.H ? 0 : 1, h = hh - kv * p.H;
             size_t drow = 0;
             float sg = 1.0f;
@@ -218,13 +245,13 @@ __device__ void epilogue(PCtx &c)
             }
 #pragma unroll 1
             for (int q = 0; q < 4; ++q) {
-                uint32_t v[32];
-                ptx::tmem_ld32(tbase + b * 256 + half * 128 + q * 32, v);
+                uint32_t d[32];
+                ptx::tmem_ld32(tbase + b * 256 + col * 128 + q * 32, d);
                 ptx::tmem_wait_ld();
                 uint32_t w[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                    w[i] = bf16x2_bits(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                    w[i] = bf16x2_bits(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1]));
                 if (!valid) continue;
                 if (p.mode == 0) {
                     uint4 *dst = reinterpret_cast<uint4 *>(kv ? p.v_out : p.k_out) +
@@ -266,6 +293,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
     c.pair = blockIdx.x >> 1;
     c.nk = p.hidden / PK;
     c.n_tiles = (p.M + 2 * PM - 1) / (2 * PM) * p.H;
+    c.n_full = c.n_tiles / p.n_pairs * p.n_pairs;
+    c.n_items = 2 * (c.n_tiles - c.n_full) <= p.n_pairs ? c.n_full + 2 * (c.n_tiles - c.n_full)
+                                                        : c.n_tiles;
+    if (c.n_items == c.n_tiles) c.n_full = c.n_tiles;
     c.lead_bar = ptx::mapa(ptx::smem_u32(&c.ctl->bar[0]), 0);
     c.peer_abort = ptx::mapa(ptx::smem_u32(&c.ctl->abort), c.rank ^ 1u);
     const int warp = threadIdx.x >> 5;
