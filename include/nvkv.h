@@ -249,7 +249,9 @@ NVKV_API nvkv_status nvfp4_kv_append(const nvkv_desc *desc, const nvkv_cache *ca
  * results as nvfp4_kv_append; cache->amax is ignored and may be NULL.
  *  - B * H must be <= 256, else NVKV_ERR_UNSUPPORTED.
  *  - The first call on a device sets up the array's address for that device
- *    (with that device current); make it before any stream capture.
+ *    (with that device current) and keeps it for the process; make it before
+ *    any stream capture.  After a cudaDeviceReset of that device the kept
+ *    address is stale: do not call this entry point on that device again.
  *  - All calls share the array: a scale-fixing first append clears it before
  *    use; calls whose work overlaps on the GPU race on it, so serialise them. */
 NVKV_API nvkv_status nvfp4_kv_append_noalloc(const nvkv_desc *desc, const nvkv_cache *cache,

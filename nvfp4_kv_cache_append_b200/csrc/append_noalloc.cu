@@ -12,15 +12,20 @@
 // until the process exits).  It calls no cudaMalloc / cudaFree.
 //
 // Limits and rules:
-//  - at most NVKV_NOALLOC_MAX_HEADS (b, h) pairs: B * H <= 256
+//  - at most 256 (b, h) pairs: B * H <= 256
 //    (2 * 256 words = 2 KiB of scratch);
 //  - the first call on each device looks up the array's device address
-//    (cudaGetSymbolAddress) with that device current; make that first call
-//    before any stream capture;
+//    (cudaGetSymbolAddress) with that device current and keeps it for the
+//    process; make that first call before any stream capture.  A
+//    cudaDeviceReset of that device invalidates the kept address (the module
+//    may load elsewhere in the new context): do not call this entry point
+//    again on that device after a reset;
 //  - every call on a device shares the one array and leaves its last contents
 //    there; a scale-fixing (first) append clears it before use.  Calls whose
 //    work overlaps on the GPU (two streams, or two threads) race on it:
 //    serialise them.
+// Validation, slot assignment, the launch and the ring update are those of
+// nvfp4_kv_append (the shared host path), with the array as the scratch.
 #include <mutex>
 
 #include "nvkv_internal.h"
@@ -54,55 +59,16 @@ cudaError_t scratch_for_current_device(uint32_t **out)
     return cudaSuccess;
 }
 
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
 
 extern "C" nvkv_status nvfp4_kv_append_noalloc(const nvkv_desc *desc, const nvkv_cache *cache,
                                                nvkv_ring *ring, const void *k, const void *v,
                                                nvkv_stream stream)
 {
-    if (!desc || !ring) return NVKV_ERR_INVALID_ARG;
-    if (desc->magic != NVKV_MAGIC || desc->version != NVKV_VERSION) return NVKV_ERR_STATE;
-    if (desc->kv_dtype != NVKV_KV_NVFP4) return NVKV_ERR_STATE;
+    if (!desc) return NVKV_ERR_INVALID_ARG;
     if ((int64_t)desc->B * desc->H > kMaxHeads) return NVKV_ERR_UNSUPPORTED;
-    if (!cache || !k || !v || !cache->k_data || !cache->v_data || !cache->k_scales ||
-        !cache->v_scales || !cache->s_g)
-        return NVKV_ERR_INVALID_ARG;
-    if (!aligned16(k) || !aligned16(v) || !aligned16(cache->k_data) ||
-        !aligned16(cache->v_data) || !aligned16(cache->k_scales) || !aligned16(cache->v_scales))
-        return NVKV_ERR_ALIGNMENT;
-
-    // the ring update an append performs, on a copy (validates desc and ring)
-    nvkv_ring next = *ring;
-    int32_t slots[NVKV_MAX_BATCH * NVKV_MAX_CHUNK];
-    const int first = ring->scales_fixed ? 0 : 1;
-    nvkv_status st = nvkv_ring_push_chunk(desc, &next, slots);
-    if (st != NVKV_OK) return st;
-
     uint32_t *scratch = nullptr;
     if (scratch_for_current_device(&scratch) != cudaSuccess) return NVKV_ERR_CUDA;
-
-    nvkv::AppendLaunch a{};
-    for (int i = 0; i < desc->B * desc->C; ++i) a.slot[i] = slots[i];
-    a.k = k;
-    a.v = v;
-    a.k_data = cache->k_data;
-    a.v_data = cache->v_data;
-    a.k_scales = cache->k_scales;
-    a.v_scales = cache->v_scales;
-    a.amax = scratch;                 // cleared by the launcher when first != 0
-    a.s_g = cache->s_g;
-    a.B = desc->B;
-    a.H = desc->H;
-    a.T = desc->grid_h * desc->grid_w;
-    a.Lq = desc->C * a.T;
-    a.Ts = nvkv::shard_tokens(desc);
-    a.tok_off = nvkv::shard_first_token(desc);
-    a.R = a.Ts * (desc->S + desc->W);
-    a.C = desc->C;
-    a.first = first;
-    if (nvkv::launch_nvfp4_append(a, (cudaStream_t)stream) != cudaSuccess) return NVKV_ERR_CUDA;
-    *ring = next;
-    return NVKV_OK;
+    // the launcher clears the scratch before a scale-fixing append uses it
+    return nvkv::nvfp4_append_with_scratch(desc, cache, ring, k, v, (cudaStream_t)stream, scratch);
 }

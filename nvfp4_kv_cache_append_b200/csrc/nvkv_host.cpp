@@ -138,9 +138,11 @@ bool newest_chunk_slots(const nvkv_desc *d, const nvkv_ring *r, int32_t *slot_ou
 // (advance = the ring), or, with advance = null, in-place overwrite of the
 // newest chunk: same slots, ring unchanged; while the first chunk is the only
 // one appended, its overwrite fixes s_g again from the new values.
+// amax_scratch: when not null, the NVFP4 amax scratch to use in place of
+// cache->amax (which may then be null).
 nvkv_status append_common(const nvkv_desc *desc, const nvkv_cache *cache, const nvkv_ring *ring,
                           nvkv_ring *advance, const void *k, const void *v, cudaStream_t stream,
-                          int dtype)
+                          int dtype, uint32_t *amax_scratch = nullptr)
 {
     const bool overwrite = advance == nullptr;
     nvkv_status st = check_desc(desc);
@@ -148,8 +150,8 @@ nvkv_status append_common(const nvkv_desc *desc, const nvkv_cache *cache, const 
     if (desc->kv_dtype != dtype) return NVKV_ERR_STATE;
     if ((st = check_ring(desc, ring)) != NVKV_OK) return st;
     if (!cache || !k || !v || !cache->k_data || !cache->v_data) return NVKV_ERR_INVALID_ARG;
-    if (dtype == NVKV_KV_NVFP4 &&
-        (!cache->k_scales || !cache->v_scales || !cache->amax || !cache->s_g))
+    uint32_t *amax = amax_scratch ? amax_scratch : cache->amax;
+    if (dtype == NVKV_KV_NVFP4 && (!cache->k_scales || !cache->v_scales || !amax || !cache->s_g))
         return NVKV_ERR_INVALID_ARG;
     if (!aligned16(k) || !aligned16(v) || !aligned16(cache->k_data) || !aligned16(cache->v_data) ||
         (dtype == NVKV_KV_NVFP4 && (!aligned16(cache->k_scales) || !aligned16(cache->v_scales))))
@@ -167,7 +169,7 @@ nvkv_status append_common(const nvkv_desc *desc, const nvkv_cache *cache, const 
     a.v_data = cache->v_data;
     a.k_scales = cache->k_scales;
     a.v_scales = cache->v_scales;
-    a.amax = cache->amax;
+    a.amax = amax;
     a.s_g = cache->s_g;
     a.B = desc->B;
     a.H = desc->H;
@@ -296,6 +298,13 @@ nvkv_status attention_common(const nvkv_desc *desc, const nvkv_cache *cache,
 }
 
 }  // namespace
+
+nvkv_status nvkv::nvfp4_append_with_scratch(const nvkv_desc *desc, const nvkv_cache *cache,
+                                            nvkv_ring *ring, const void *k, const void *v,
+                                            cudaStream_t stream, uint32_t *amax_scratch)
+{
+    return append_common(desc, cache, ring, ring, k, v, stream, NVKV_KV_NVFP4, amax_scratch);
+}
 
 extern "C" {
 

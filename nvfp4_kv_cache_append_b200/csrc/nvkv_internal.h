@@ -32,6 +32,12 @@ inline int shard_tokens(const nvkv_desc *d)
 inline int shard_first_token(const nvkv_desc *d) { return d->shard_rank * shard_tokens(d); }
 
 cudaError_t launch_nvfp4_append(const AppendLaunch &a, cudaStream_t s);
+// nvfp4_kv_append with its amax scratch given by the caller (amax_scratch
+// replaces cache->amax, which may be null): the same checks, slots, launch
+// and ring update.
+nvkv_status nvfp4_append_with_scratch(const nvkv_desc *desc, const nvkv_cache *cache,
+                                      nvkv_ring *ring, const void *k, const void *v,
+                                      cudaStream_t stream, uint32_t *amax_scratch);
 cudaError_t launch_bf16_append(const AppendLaunch &a, cudaStream_t s);
 cudaError_t launch_encode_e2m1(const float *y, uint8_t *codes, size_t n, cudaStream_t s);
 cudaError_t launch_encode_block_scale(const float *t, uint8_t *codes, size_t n, cudaStream_t s);

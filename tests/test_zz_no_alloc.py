@@ -18,9 +18,10 @@ import kvsynth
 pytestmark = pytest.mark.gpu
 
 
-def _pair(wl):
+def _pair(wl, shard=(0, 1)):
     import nvfp4_kv_cache_append_b200 as nv
-    mk = lambda: nv.KVCache(wl.B, wl.H, wl.grid_h, wl.grid_w, wl.C, wl.S, wl.W, nv.NVKV_KV_NVFP4)
+    mk = lambda: nv.KVCache(wl.B, wl.H, wl.grid_h, wl.grid_w, wl.C, wl.S, wl.W, nv.NVKV_KV_NVFP4,
+                            shard_rank=shard[0], shard_count=shard[1])
     return mk(), mk()
 
 
@@ -55,6 +56,32 @@ def test_noalloc_matches_regular_append(name):
             torch.cuda.synchronize()
             _same(ref, new)
         assert int(new.amax.sum()) == 0     # the caller's amax plane was never used
+
+
+def _two_appends(nv, wl, shard=(0, 1)):
+    ref, new = _pair(wl, shard)
+    for step in (1, 2):
+        x = kvsynth.chunk_qkv(wl, step, 0)
+        k, v = x["k"].cuda(), x["v"].cuda()
+        ref.append(k, v)
+        _noalloc_append(nv, new, k, v)
+        torch.cuda.synchronize()
+        _same(ref, new)
+    assert int(new.amax.sum()) == 0
+
+
+def test_noalloc_at_the_head_limit():
+    """B * H = 256: the scratch array's last word is in use."""
+    import nvfp4_kv_cache_append_b200 as nv
+    wl = kvsynth.Workload(name="heads256", B=4, H=64, D=128, grid_h=4, grid_w=4, C=1, S=1, W=3, steps=2)
+    _two_appends(nv, wl)
+
+
+@pytest.mark.parametrize("rank", [0, 1])
+def test_noalloc_shard(rank):
+    """A shard of a two-way sequence-parallel KV split."""
+    import nvfp4_kv_cache_append_b200 as nv
+    _two_appends(nv, kvsynth.WORKLOADS["tiny"], shard=(rank, 2))
 
 
 def test_noalloc_rejects_too_many_heads():
