@@ -36,6 +36,7 @@ namespace {
 
 using namespace q4;
 
+
 __device__ __forceinline__ uint4 ld_stream(const uint4 *p)
 {
     uint4 r;
@@ -83,6 +84,32 @@ __global__ void k_first_chunk_amax(const uint4 *__restrict__ k, const uint4 *__r
     if (tid < H && s_max[tid]) atomicMax(&amax[(t * B + b) * H + tid], s_max[tid]);
 }
 
+// Quantize the two blocks (elements 32 pair .. 32 pair + 31) of one
+// token-head row given as four 16-byte words, and write codes and scales
+// into cache row `row`.
+__device__ __forceinline__ void quantize_pair(const AppendLaunch &a, int t, int h, int pr,
+                                              size_t row, float sg, uint4 w0, uint4 w1, uint4 w2,
+                                              uint4 w3)
+{
+    uint2 c0, c1;
+    const uint32_t s0 = quantize_block(w0, w1, sg, c0);
+    const uint32_t s1 = quantize_block(w2, w3, sg, c1);
+    *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(t ? a.v_data : a.k_data) + row * 64 + pr * 16) =
+        make_uint4(c0.x, c0.y, c1.x, c1.y);
+    *reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(t ? a.v_scales : a.k_scales) + row * 8 +
+                                  pr * 2) = (uint16_t)(s0 | (s1 << 8));
+}
+
+__device__ __forceinline__ float head_scale(const AppendLaunch &a, int gi, bool writer)
+{
+    if (a.first) {
+        const float sg = global_scale_from_amax(a.amax[gi]);
+        if (writer) a.s_g[gi] = sg;
+        return sg;
+    }
+    return a.s_g[gi];
+}
+
 // blockDim = (4H, ty): threadIdx.x = h * 4 + pair (blocks 2 pair, 2 pair + 1
 // of the token-head: 64 bytes in, 16 code bytes and 2 scale bytes out),
 // threadIdx.y = token in the CTA's token group.  grid = (ceil(C Ts / ty), 2B):
@@ -100,25 +127,11 @@ __global__ void __launch_bounds__(512) k_nvfp4_append(const __grid_constant__ Ap
                        (((size_t)b * a.Lq + src_l) * a.H + h) * 16 + pr * 4;
     const uint4 w0 = ld_stream(src), w1 = ld_stream(src + 1);
     const uint4 w2 = ld_stream(src + 2), w3 = ld_stream(src + 3);
-
     const int gi = (t * a.B + b) * a.H + h;
-    float sg;
-    if (a.first) {
-        sg = global_scale_from_amax(a.amax[gi]);
-        if (l == 0 && pr == 0) a.s_g[gi] = sg;
-    } else {
-        sg = a.s_g[gi];
-    }
-    uint2 c0, c1;
-    const uint32_t s0 = quantize_block(w0, w1, sg, c0);
-    const uint32_t s1 = quantize_block(w2, w3, sg, c1);
-
+    const float sg = head_scale(a, gi, l == 0 && pr == 0);
     const int slot = a.slot[b * a.C + frame];
-    const size_t row = (size_t)(b * a.H + h) * a.R + (size_t)slot * a.Ts + tok;
-    *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(t ? a.v_data : a.k_data) + row * 64 + pr * 16) =
-        make_uint4(c0.x, c0.y, c1.x, c1.y);
-    *reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(t ? a.v_scales : a.k_scales) + row * 8 +
-                                  pr * 2) = (uint16_t)(s0 | (s1 << 8));
+    quantize_pair(a, t, h, pr, (size_t)(b * a.H + h) * a.R + (size_t)slot * a.Ts + tok, sg, w0, w1,
+                  w2, w3);
 }
 
 // bf16 twin: blockDim = (16H, ty), one 16-byte chunk per thread; rows as in
@@ -171,7 +184,6 @@ cudaError_t launch_nvfp4_append(const AppendLaunch &a_in, cudaStream_t s)
     AppendLaunch a = a_in;
     a.inv_Ts = 1.0f / (float)a.Ts;
     const dim3 blk = append_block(a.H, 4);
-    const dim3 grid((a.C * a.Ts + blk.y - 1) / blk.y, 2 * a.B);
     if (a.first) {
         cudaError_t e = cudaMemsetAsync(a.amax, 0, sizeof(uint32_t) * 2 * a.B * a.H, s);
         if (e != cudaSuccess) return e;
@@ -182,6 +194,7 @@ cudaError_t launch_nvfp4_append(const AppendLaunch &a_in, cudaStream_t s)
                                               static_cast<const uint4 *>(a.v), a.amax, a.B, a.H,
                                               a.Lq);
     }
+    const dim3 grid((a.C * a.Ts + blk.y - 1) / blk.y, 2 * a.B);
     k_nvfp4_append<<<grid, blk, 0, s>>>(a);
     return cudaGetLastError();
 }

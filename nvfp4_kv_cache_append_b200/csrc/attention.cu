@@ -735,26 +735,30 @@ __device__ void mma_role(Ctx &c)
     const uint32_t vs = c.sbase + OFF_V;
     const uint16_t both = 0x3;
 
+    // Shared-memory descriptors: the start address (>> 4) is the low field,
+    // so the descriptor of base + off is desc(base) + off / 16 (all of shared
+    // memory lies below 2^18 bytes, so the field cannot carry).  Built once,
+    // they leave the issuing thread two adds per MMA.
+    const uint64_t dk0 = ptx::smem_desc_sw128(ks, 16, 1024);
+    const uint64_t dv0 = ptx::smem_desc_sw128(vs, V_TILE, 1024);
     // S_buf = Q K^T: A = Q (TMEM, 8 x 16 channels), B = the K halves, K-major
     auto issue_s = [&](int buf, int kb) {
-        const uint32_t kt = ks + kb * K_TILE;
+        const uint64_t dk = dk0 + (uint64_t)(kb * (K_TILE >> 4));
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
             ptx::mma2_f16_ts(tmem + TM_S + buf * 128, tmem + TM_Q + kk * 8,
-                             ptx::smem_desc_sw128(kt + (kk >> 2) * K_HALF + (kk & 3) * 32, 16,
-                                                  1024),
-                             idS, kk > 0);
+                             dk + (uint64_t)(((kk >> 2) * K_HALF + (kk & 3) * 32) >> 4), idS,
+                             kk > 0);
         ptx::mma2_commit_mc(&c.ctl->bar[B_S + buf], both);
         ptx::mma2_commit_mc(&c.ctl->bar[B_KFREE + kb], both);
     };
     // O += P V: A = P (TMEM over S_buf, 8 x 16 keys), B = the V halves, MN-major
     auto issue_pv = [&](int buf, int vb, bool first) {
-        const uint32_t vt = vs + vb * V_TILE;
+        const uint64_t dv = dv0 + (uint64_t)(vb * (V_TILE >> 4));
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
             ptx::mma2_f16_ts(tmem + TM_O, tmem + TM_S + buf * 128 + kk * 8,
-                             ptx::smem_desc_sw128(vt + kk * 2048, V_TILE, 1024), idO,
-                             (!first || kk > 0) ? 1u : 0u);
+                             dv + (uint64_t)(kk * (2048 >> 4)), idO, (!first || kk > 0) ? 1u : 0u);
         ptx::mma2_commit_mc(&c.ctl->bar[B_VFREE + vb], both);
     };
 
