@@ -143,6 +143,196 @@ def bench_config(wl, kv, ws):
 
 # --------------------------------------------------------------- our arm
 
+class StreamBench:
+    """Steady-state AR steps of one workload on this GPU: evict + append +
+    attention per step, over N_LAYERS independent caches and input sets
+    cycled (one cache for the long run), inputs resident in HBM."""
+
+    def __init__(self, nv, torch, wl, kvd, seed, stream):
+        import kvsynth
+        self.nv, self.torch, self.wl, self.stream = nv, torch, wl, stream
+        self.n_layers = 1 if wl.name == "long600" else N_LAYERS
+        self.sets = []
+        for i in range(N_LAYERS):
+            x = kvsynth.chunk_qkv(wl, 1000 + i, seed=seed)
+            self.sets.append({k: v.cuda() for k, v in x.items()})
+        self.caches = [nv.KVCache(wl.B, wl.H, wl.grid_h, wl.grid_w, wl.C, wl.S, wl.W, kvd)
+                       for _ in range(self.n_layers)]
+        self.outs = [torch.empty_like(self.sets[0]["q"]) for _ in range(self.n_layers)]
+        # multi-shot streams: shot ids per AR step (per-shot sinks, masking)
+        self.sched = kvsynth.shot_schedule(wl, seed) if wl.shots > 1 else None
+        self.steps_done = [0] * self.n_layers
+        # fill every ring to steady state (window full); multi-shot runs start
+        # their shot schedule at the first step
+        fill = 0 if self.sched is not None else (wl.S + wl.W) // wl.C
+        for li in range(self.n_layers):
+            for s_ in range(fill):
+                x = self.sets[s_ % N_LAYERS]
+                c = self.begin_step(li)
+                c.append(x["k"], x["v"])
+                c.attention(x["q"], out=self.outs[li])
+        torch.cuda.synchronize()
+
+    def shot_ids(self, li):
+        if self.sched is None:
+            return None
+        # the schedule repeats; shot ids keep increasing across repeats
+        n = len(self.sched[0])
+        k, rep = self.steps_done[li] % n, self.steps_done[li] // n
+        return [self.sched[b][k] + self.wl.shots * rep for b in range(self.wl.B)]
+
+    def begin_step(self, li):
+        c = self.caches[li]
+        ids = self.shot_ids(li)
+        if ids is not None:
+            for b, sid in enumerate(ids):
+                c.begin_shot(b, sid)
+        self.steps_done[li] += 1
+        need = self.wl.C - min(c.free_frames(b) for b in range(self.wl.B))
+        if need > 0:
+            c.evict(need)
+        return c
+
+    def run(self, steps, warmup, dist=None, clocks=None):
+        """Device-timed steps: events around the whole loop and around each
+        step's append and attention (all on one stream)."""
+        torch, wl, stream = self.torch, self.wl, self.stream
+        ev = lambda: torch.cuda.Event(enable_timing=True)
+        visible = []
+
+        def one_step(i, timing):
+            li = i % self.n_layers
+            x = self.sets[(i + 1) % N_LAYERS]
+            e0 = e1 = e2 = None
+            if timing:
+                e0 = ev(); e0.record(stream)
+            c = self.begin_step(li)
+            c.append(x["k"], x["v"], stream=stream)
+            if timing:
+                e1 = ev(); e1.record(stream)
+            c.attention(x["q"], out=self.outs[li], stream=stream)
+            if timing:
+                e2 = ev(); e2.record(stream)
+                visible.append(sum(len(c.visible(b)[2]) for b in range(wl.B)) * wl.T)
+            return e0, e1, e2
+
+        for i in range(warmup):
+            one_step(i, False)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        foot0 = [c.footprint_bytes() for c in self.caches]
+        alloc0 = torch.cuda.memory_allocated()
+        free0 = torch.cuda.mem_get_info()[0]
+        if clocks is not None:
+            clocks.start()
+            time.sleep(0.3)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        t0, t1 = ev(), ev()
+        t0.record(stream)
+        marks = [one_step(warmup + i, True) for i in range(steps)]
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        clk = clocks.stop() if clocks is not None else None
+        for c in self.caches:
+            assert c.device_status() == 0, "device-side pipeline error"
+        app = [a.elapsed_time(b) for a, b, _ in marks]
+        att = [b.elapsed_time(c) for _, b, c in marks]
+        step = [a.elapsed_time(c) for a, _, c in marks]
+        return {"total_ms": t0.elapsed_time(t1), "app_ms": app, "att_ms": att, "step_ms": step,
+                "visible_keys": visible, "clocks": clk,
+                "memory": {"cache_footprint_bytes": foot0[0],
+                           "footprint_constant": [c.footprint_bytes() for c in self.caches] == foot0,
+                           "allocated_delta_bytes": torch.cuda.memory_allocated() - alloc0,
+                           "device_free_delta_bytes": torch.cuda.mem_get_info()[0] - free0}}
+
+
+def _pct(xs, p):
+    xs = sorted(xs)
+    return xs[min(len(xs) - 1, int(p * len(xs)))]
+
+
+def cold_append_us(nv, torch, wl, kvd, n=40, reps=5):
+    """Isolated cold-L2 time of one steady-state append launch (s_g fixed),
+    by difference: events around n x (256 MB L2 flush + append) and around
+    n x flush, so launch gaps hide behind the flush writes; median of reps.
+    The append runs as an in-place overwrite of the newest chunk, which
+    launches the same kernel on the same slots without moving the ring."""
+    import kvsynth
+    x = {k: v.cuda() for k, v in kvsynth.chunk_qkv(wl, 1000, 0).items()}
+    c = nv.KVCache(wl.B, wl.H, wl.grid_h, wl.grid_w, wl.C, wl.S, wl.W, kvd)
+    for _ in range(2):
+        c.append(x["k"], x["v"])
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def loop(with_append):
+        a, b = ev(), ev()
+        torch.cuda.synchronize()
+        a.record()
+        for i in range(n):
+            flush.fill_(i & 255)
+            if with_append:
+                c.overwrite(x["k"], x["v"])
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) * 1e3 / n
+
+    loop(True), loop(False)
+    res = sorted(loop(True) - loop(False) for _ in range(reps))
+    assert c.device_status() == 0, "device-side pipeline error"
+    return res[len(res) // 2]
+
+
+def workload_summary(nv, torch, wl, kvd, steps, warmup, stream, peaks, seed=0):
+    """One short steady-state run of another workload: attention TFLOP/s over
+    the visible keys, append GB/s (in the step and isolated cold), step
+    latency percentiles."""
+    num = workload_numbers(wl)
+    fp4 = kvd == nv.NVKV_KV_NVFP4
+    sb = StreamBench(nv, torch, wl, kvd, seed, stream)
+    r = sb.run(steps, warmup)
+    K = len(r["att_ms"])
+    flop = 4.0 * wl.H * wl.Lq * 128 * (sum(r["visible_keys"]) / K)
+    att = sum(r["att_ms"]) / K
+    app = sum(r["app_ms"]) / K
+    tfl = flop / (att / 1e3) / 1e12
+    app_bytes = num["append_bytes"] if fp4 else num["twin_append_bytes"]
+    out = {"workload": bench_config(wl, "nvfp4" if fp4 else "bf16", 1)["workload"],
+           "steps": K, "attn_ms": att, "attn_tflops": tfl,
+           "attn_frac": tfl / peaks["bf16_tflops"],
+           "append_in_step_gbs": app_bytes / (app / 1e3) / 1e9,
+           "step_ms_p50": _pct(r["step_ms"], 0.5), "step_ms_p99": _pct(r["step_ms"], 0.99)}
+    if wl.shots > 1:
+        # steps differ in work (a shot start sees 7 of 21 frames per stream):
+        # the latency per visible key is the flat quantity
+        per = [1e6 * t / v for t, v in zip(r["step_ms"], r["visible_keys"])]
+        out["step_ns_per_visible_key_p50"] = _pct(per, 0.5)
+        out["step_ns_per_visible_key_p99"] = _pct(per, 0.99)
+        out["visible_keys_per_step_min_max"] = [min(r["visible_keys"]), max(r["visible_keys"])]
+    if wl.name == "long600":
+        out["memory"] = r["memory"]
+    if wl.name != "long600":
+        us = cold_append_us(nv, torch, wl, kvd)
+        out["append_cold_us"] = us
+        out["append_cold_gbs"] = app_bytes / (us / 1e6) / 1e9
+        out["append_cold_frac"] = out["append_cold_gbs"] / peaks["hbm_gbs"]
+    del sb
+    torch.cuda.empty_cache()
+    return out
+
+
+# Other workloads reported beside the headline (one GPU only): the 5B-like
+# stream, the bf16-KV twin on both streams, the multi-shot batch, and the
+# 600-step stream's latency and allocation record.
+EXTRA_RUNS = [("stream5b", "nvfp4", 60), ("stream1p3b", "bf16", 60), ("stream5b", "bf16", 60),
+              ("multishot", "nvfp4", 96), ("long600", "nvfp4", 300)]
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -162,124 +352,34 @@ def run_ours(args):
     stream = torch.cuda.Stream()
     torch.cuda.set_stream(stream)
 
-    # inputs: seeded sets, resident in HBM before timing; one cache per
-    # emulated layer (one cache for the long run: 600 steps of one stream)
-    n_layers = 1 if wl.name == "long600" else N_LAYERS
-    sets = []
-    for i in range(N_LAYERS):
-        x = kvsynth.chunk_qkv(wl, 1000 + i, seed=rank)
-        sets.append({k: v.cuda() for k, v in x.items()})
-    caches = [nv.KVCache(wl.B, wl.H, wl.grid_h, wl.grid_w, wl.C, wl.S, wl.W, kvd)
-              for _ in range(n_layers)]
-    outs = [torch.empty_like(sets[0]["q"]) for _ in range(n_layers)]
-    # multi-shot streams: shot ids per AR step (per-shot sinks, masking)
-    sched = kvsynth.shot_schedule(wl, rank) if wl.shots > 1 else None
-    steps_done = [0] * n_layers
-
-    def begin_step(li):
-        c = caches[li]
-        if sched is not None:
-            # the schedule repeats; shot ids keep increasing across repeats
-            n = len(sched[0])
-            k, rep = steps_done[li] % n, steps_done[li] // n
-            for b in range(wl.B):
-                c.begin_shot(b, sched[b][k] + wl.shots * rep)
-        steps_done[li] += 1
-        need = wl.C - min(c.free_frames(b) for b in range(wl.B))
-        if need > 0:
-            c.evict(need)
-        return c
-
-    # fill every ring to steady state (window full); multi-shot runs start
-    # their shot schedule at the first step
-    fill = 0 if sched is not None else (wl.S + wl.W) // wl.C
-    for li in range(n_layers):
-        for s_ in range(fill):
-            x = sets[s_ % N_LAYERS]
-            c = begin_step(li)
-            c.append(x["k"], x["v"])
-            c.attention(x["q"], out=outs[li])
-    torch.cuda.synchronize()
-
-    ev = lambda: torch.cuda.Event(enable_timing=True)
-    visible_keys = []          # per timed step: sum over streams of visible keys
-
-    def one_step(i, timing):
-        li = i % n_layers
-        x = sets[(i + 1) % N_LAYERS]
-        e0 = e1 = e2 = None
-        if timing:
-            e0 = ev(); e0.record(stream)
-        c = begin_step(li)
-        c.append(x["k"], x["v"], stream=stream)
-        if timing:
-            e1 = ev(); e1.record(stream)
-        c.attention(x["q"], out=outs[li], stream=stream)
-        if timing:
-            e2 = ev(); e2.record(stream)
-            visible_keys.append(sum(len(c.visible(b)[2]) for b in range(wl.B)) * wl.T)
-        return e0, e1, e2
-
-    for i in range(args.warmup):
-        one_step(i, False)
-    torch.cuda.synchronize()
-    if ws > 1:
-        dist.barrier()
-    foot0 = [c.footprint_bytes() for c in caches]
-    alloc0 = torch.cuda.memory_allocated()
-    free0 = torch.cuda.mem_get_info()[0]
+    sb = StreamBench(nv, torch, wl, kvd, rank, stream)
     clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
-    torch.cuda.synchronize()
-    if ws > 1:
-        dist.barrier()
-    t_start, t_end = ev(), ev()
-    t_start.record(stream)
-    marks = [one_step(args.warmup + i, True) for i in range(args.steps)]
-    t_end.record(stream)
-    torch.cuda.synchronize()
-    if ws > 1:
-        dist.barrier()
-    clk = clocks.stop()
-    total_ms = t_start.elapsed_time(t_end)
-    app_ms = [a.elapsed_time(b) for a, b, _ in marks]
-    att_ms = [b.elapsed_time(c) for _, b, c in marks]
-    step_ms = sorted(a.elapsed_time(c) for a, _, c in marks)
-    memory = {"cache_footprint_bytes": foot0[0],
-              "footprint_constant": [c.footprint_bytes() for c in caches] == foot0,
-              "allocated_delta_bytes": torch.cuda.memory_allocated() - alloc0,
-              "device_free_delta_bytes": torch.cuda.mem_get_info()[0] - free0}
+    r = sb.run(args.steps, args.warmup, dist if ws > 1 else None, clocks)
+    clk = r["clocks"]
+    total_ms = r["total_ms"]
     if ws > 1:
         t = torch.tensor([total_ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
-    for c in caches:
-        assert c.device_status() == 0, "device-side pipeline error"
 
     # end to end through the public host pipeline: every step uploads its
     # q/k/v from pinned host memory, runs evict + append + attention and
     # downloads the output to pinned host memory, on three streams so that
     # step k's upload overlaps step k-1's compute and step k-2's download
-    host = [{k: v.cpu().pin_memory() for k, v in s.items()} for s in sets]
-    host_out = [torch.empty(sets[0]["q"].shape, dtype=torch.bfloat16).pin_memory()
+    host = [{k: v.cpu().pin_memory() for k, v in s_.items()} for s_ in sb.sets]
+    host_out = [torch.empty(sb.sets[0]["q"].shape, dtype=torch.bfloat16).pin_memory()
                 for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host[0].values())
     d2h = host_out[0].numel() * host_out[0].element_size()
     # one set of streams for all emulated layers: their steps run in order,
     # as a model's layers would
     pstreams = tuple(torch.cuda.Stream() for _ in range(3))
-    pipes = [nv.HostPipeline(c, streams=pstreams) for c in caches]
+    pipes = [nv.HostPipeline(c, streams=pstreams) for c in sb.caches]
 
     def e2e_step(i):
-        li = i % n_layers
-        if sched is not None:
-            n = len(sched[0])
-            k, rep = steps_done[li] % n, steps_done[li] // n
-            shot = [sched[b][k] + wl.shots * rep for b in range(wl.B)]
-        else:
-            shot = None
-        steps_done[li] += 1
+        li = i % sb.n_layers
+        shot = sb.shot_ids(li)
+        sb.steps_done[li] += 1
         x = host[(i + 1) % N_LAYERS]
         pipes[li].submit(x["q"], x["k"], x["v"], host_out[i & 1], shot=shot)
 
@@ -290,6 +390,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     if ws > 1:
         dist.barrier()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
     a, b = ev(), ev()
     a.record(pstreams[0])
     for i in range(args.steps):
@@ -301,7 +402,7 @@ def run_ours(args):
         t = torch.tensor([e2e_ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
-    for c in caches:
+    for c in sb.caches:
         assert c.device_status() == 0, "device-side pipeline error"
 
     peaks = _peaks()
@@ -309,14 +410,15 @@ def run_ours(args):
     ms_step = total_ms / K
     tok_per_step = wl.B * wl.Lq
     value = ws * tok_per_step * K / (total_ms / 1e3)
-    att_avg = sum(att_ms) / K
-    app_avg = sum(app_ms) / K
+    att_avg = sum(r["att_ms"]) / K
+    app_avg = sum(r["app_ms"]) / K
     # FLOP of the steps actually timed: visible keys only (multi-shot masks)
-    flop_step = 4.0 * wl.H * wl.Lq * 128 * (sum(visible_keys) / K)
+    flop_step = 4.0 * wl.H * wl.Lq * 128 * (sum(r["visible_keys"]) / K)
     attn_tflops = flop_step / (att_avg / 1e3) / 1e12
     app_bytes = num["append_bytes"] if fp4 else num["twin_append_bytes"]
     append_gbs = app_bytes / (app_avg / 1e3) / 1e9
     peak = peaks["bf16_tflops_sustained"] if K * ms_step > 2000 else peaks["bf16_tflops"]
+    del pipes
     line = {
         "metric": METRIC,
         "value": value,
@@ -333,9 +435,8 @@ def run_ours(args):
         "config": bench_config(wl, args.kv, ws),
         "attn_tflops": attn_tflops,
         "attn_flop_per_step": flop_step,
-        "step_ms": {"p50": step_ms[len(step_ms) // 2],
-                    "p99": step_ms[min(len(step_ms) - 1, int(0.99 * len(step_ms)))]},
-        "memory": memory,
+        "step_ms": {"p50": _pct(r["step_ms"], 0.5), "p99": _pct(r["step_ms"], 0.99)},
+        "memory": r["memory"],
         "attn_ms": att_avg,
         "append_gbs": append_gbs,
         "append_ms": app_avg,
@@ -343,13 +444,36 @@ def run_ours(args):
                      "unit": "TFLOP/s", "frac": attn_tflops / peak,
                      "traffic": _ncu_traffic("k_chunk_attn<1, 0>", wl.name) if fp4 else None,
                      "kernel": "k_chunk_attn", "peak_source": peaks["source"] + " bf16 (f16 same nominal rate)"},
-        "append_roofline": {"bound": "hbm", "achieved": append_gbs, "peak": peaks["hbm_gbs"],
-                            "unit": "GB/s", "frac": append_gbs / peaks["hbm_gbs"]},
+        "append_roofline_in_step": {"bound": "hbm", "achieved": append_gbs, "peak": peaks["hbm_gbs"],
+                                    "unit": "GB/s", "frac": append_gbs / peaks["hbm_gbs"],
+                                    "timing": "events around the append inside the timed steps"},
         "e2e": {"value": ws * tok_per_step * K / (e2e_ms / 1e3), "unit": "query tok/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * K,
         "clocks": clk,
     }
+    del sb
+    torch.cuda.empty_cache()
+    if ws == 1 and wl.name != "long600":
+        us = cold_append_us(nv, torch, wl, kvd)
+        gbs = app_bytes / (us / 1e6) / 1e9
+        line["append_roofline"] = {
+            "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": gbs / peaks["hbm_gbs"], "kernel": "k_nvfp4_append" if fp4 else "k_bf16_append",
+            "us_per_launch": us,
+            "timing": "isolated, cold L2: 40 x (256 MB flush + append) minus 40 x flush, median of 5"}
+    if ws == 1 and not args.no_extra:
+        clocks2 = ClockSampler(local)
+        clocks2.start()
+        extra = {}
+        for name, kv, steps in EXTRA_RUNS:
+            if name == wl.name and kv == args.kv:
+                continue
+            kd = nv.NVKV_KV_NVFP4 if kv == "nvfp4" else nv.NVKV_KV_BF16
+            extra[f"{name} {kv}"] = workload_summary(nv, torch, kvsynth.WORKLOADS[name], kd,
+                                                     steps, args.warmup, stream, peaks)
+        extra["clocks"] = clocks2.stop()
+        line["other_workloads"] = extra
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, seconds=args.cpu_seconds)
     if rank == 0:
@@ -724,6 +848,8 @@ def main():
     ap.add_argument("--kv", default="nvfp4", choices=["nvfp4", "bf16"])
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other workloads reported beside the headline")
     ap.add_argument("--sp-emulate", action="store_true",
                     help="per-rank kernel times of the sequence-parallel split, emulated on one GPU")
     ap.add_argument("--project", action="store_true",

@@ -115,9 +115,12 @@ typedef struct {
 } nvkv_desc;
 
 /* Device planes of one cache (caller-owned; sizes from nvkv_plane_bytes).
- * R = (S + W) * Ts rows per (batch, head), Ts = T / shard_count tokens of
- * each frame; physical frame slot p holds rows [p*Ts, (p+1)*Ts), row p*Ts + i
- * being token shard_rank*Ts + i of the frame in that slot.
+ * Ts = T / shard_count tokens of each frame are cached, in Tr = Ts rounded up
+ * to even rows per frame slot (an odd Ts adds one padding row, so that every
+ * slot's scale rows start on a 16-byte boundary); R = (S + W) * Tr rows per
+ * (batch, head).  Physical frame slot p holds rows [p*Tr, p*Tr + Ts), row
+ * p*Tr + i being token shard_rank*Ts + i of the frame in that slot; the
+ * padding row is never written, and no result depends on its contents.
  *   NVFP4: k_data/v_data = codes [B][H][R][64] u8, k_scales/v_scales = E4M3
  *          block scales [B][H][R][8] u8, amax [2][B][H] (float bits, K then
  *          V), s_g [2][B][H] f32.
@@ -185,8 +188,9 @@ NVKV_API nvkv_status nvkv_desc_init(nvkv_desc *desc, int B, int H, int grid_h, i
  *    query, the attention over the shard's keys only, with its lse; the
  *    shards' results are combined by nvkv_lse_merge.
  * NVKV_ERR_INVALID_ARG unless 1 <= count <= NVKV_MAX_SHARDS, 0 <= rank <
- * count and T is a multiple of count; NVKV_ERR_UNSUPPORTED for an NVFP4
- * desc with T/count odd.  count = 1 gives back the whole cache. */
+ * count and T is a multiple of count.  An odd T/count (1560 tokens in 8
+ * shards: 195) is fine: the slots then carry a padding row.  count = 1 gives
+ * back the whole cache. */
 NVKV_API nvkv_status nvkv_desc_set_shard(nvkv_desc *desc, int rank, int count);
 
 /* Bytes the caller must allocate for one plane (NVKV_PLANE_*) of a cache of
@@ -297,18 +301,24 @@ NVKV_API size_t nvkv_attention_workspace_bytes(const nvkv_desc *desc);
  * chunk included, in full).  Keys are read from the cache, dequantized and
  * rotated by 3D RoPE at (their frame's RoPE index, h, w); queries are rotated
  * at (the RoPE index of their own frame, h, w).  Logits use 1/sqrt(128).
+ * Any finite bf16 q is accepted: each query row is multiplied by the power of
+ * two 2^e that puts its largest |q| in [2^13, 2^14) before it is rounded to
+ * the f16 tensor-core operand, and 2^-e is folded into that row's logit
+ * scale, which leaves the logits of rows already inside f16's range
+ * unchanged bit for bit.
  * workspace: device memory of nvkv_attention_workspace_bytes() bytes (else
  * NVKV_ERR_CAPACITY).  NVKV_ERR_STATE if nothing was appended yet;
  * NVKV_ERR_UNSUPPORTED for a RoPE
- * split other than 44/42/42, grid_h or grid_w above 256, or (NVFP4) an odd
- * number of tokens per frame. */
+ * split other than 44/42/42 or grid_h or grid_w above 256. */
 NVKV_API nvkv_status chunk_attention_nvfp4kv(const nvkv_desc *desc, const nvkv_cache *cache,
                                     const nvkv_ring *ring, const void *q, void *out, float *lse,
                                     void *workspace, size_t workspace_bytes, nvkv_stream stream);
 
 /* The bf16-KV twin of chunk_attention_nvfp4kv.  Both attention calls feed the
- * tensor cores f16 operands with f32 accumulation; the twin therefore needs
- * cached K/V and rotated Q/K inside the f16 range (|x| < 65504). */
+ * tensor cores f16 operands with f32 accumulation.  Q is range-scaled per row
+ * as in chunk_attention_nvfp4kv; the twin's cached K and V are converted to
+ * f16 as they are, so they must lie inside the f16 range (|K| and |V| below
+ * 65504 after RoPE), and values below 2^-14 lose precision. */
 NVKV_API nvkv_status chunk_attention_bf16kv(const nvkv_desc *desc, const nvkv_cache *cache,
                                    const nvkv_ring *ring, const void *q, void *out, float *lse,
                                    void *workspace, size_t workspace_bytes, nvkv_stream stream);
@@ -359,6 +369,32 @@ NVKV_API nvkv_status nvfp4_kv_project_append(const nvkv_desc *desc, const nvkv_c
 NVKV_API nvkv_status nvkv_lse_merge(int n_parts, const void *const *o_parts,
                                     const float *const *lse_parts, int B, int H, int Lq, int q0,
                                     int q1, void *out, float *lse_out, nvkv_stream stream);
+
+/* One step's exchange of a sequence-parallel split: a cross-rank barrier on
+ * device flags, bounded in time, fused with nvkv_lse_merge in one kernel, so
+ * that no rank reads a peer's part before the peer has finished writing it.
+ * This rank is `rank` of n_parts ranks; o_parts, lse_parts and the result as
+ * in nvkv_lse_merge.  flags: host array of n_parts device pointers, flags[j]
+ * rank j's signal array of NVKV_MAX_SHARDS uint32 (memory this process can
+ * store to and load from: a peer mapping or symmetric memory), zero-filled on
+ * every rank before any rank's first call.  epoch: 1 on the first call, one
+ * more on each later call, the same sequence on every rank (wrap-safe).  Each
+ * CTA stores epoch into flags[j][rank] for every j (release, system scope:
+ * this rank's part, written by earlier work on `stream`, is visible to a
+ * rank that sees the value), then waits until flags[rank][j] has reached
+ * epoch for every j.  A wait longer than timeout_us, or a nonzero *status,
+ * ends it: the kernel writes NVKV_ERR_TIMEOUT to *status (if it was zero) and
+ * skips the merge (the output is undefined); nothing traps or hangs.  A rank
+ * reuses its part's memory only after its next call's barrier, by which time
+ * every rank has finished reading it.  NVKV_ERR_INVALID_ARG as nvkv_lse_merge
+ * and for a null flags entry or status, rank outside [0, n_parts), epoch 0 or
+ * timeout_us 0; NVKV_ERR_ALIGNMENT for flags or status not 4-byte aligned. */
+NVKV_API nvkv_status nvkv_lse_merge_synced(int n_parts, const void *const *o_parts,
+                                           const float *const *lse_parts,
+                                           uint32_t *const *flags, int rank, uint32_t epoch,
+                                           uint32_t timeout_us, int32_t *status, int B, int H,
+                                           int Lq, int q0, int q1, void *out, float *lse_out,
+                                           nvkv_stream stream);
 
 /* Test hook of the failure path (no counterpart in the paper).  With fault =
  * NVKV_FAULT_SKIP_FIRST_STAGE the next chunk_attention_* call on this thread

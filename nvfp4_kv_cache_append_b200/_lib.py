@@ -88,6 +88,10 @@ def _load():
         "nvfp4_kv_project_append": (i32, [D, C, R, vp, i32, vp, vp, vp, sz, vp]),
         "nvkv_lse_merge": (i32, [i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, i32,
                                  i32, vp, vp, vp]),
+        "nvkv_lse_merge_synced": (i32, [i32, ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                        ctypes.POINTER(vp), i32, ctypes.c_uint32,
+                                        ctypes.c_uint32, vp, i32, i32, i32, i32, i32, vp, vp,
+                                        vp]),
         "nvkv_plane_bytes": (sz, [D, i32]),
         "nvkv_ring_init": (i32, [D, R]),
         "kv_ring_evict": (i32, [D, R, i32]),
@@ -150,6 +154,21 @@ def nvkv_lse_merge(o_ptrs, lse_ptrs, B, H, Lq, q0, q1, out_ptr, lse_out_ptr=None
     la = (ctypes.c_void_p * max(n, 1))(*lse_ptrs)
     _check(lib.nvkv_lse_merge(n, oa, la, B, H, Lq, q0, q1, out_ptr, lse_out_ptr, stream),
            "nvkv_lse_merge")
+
+
+def nvkv_lse_merge_synced(o_ptrs, lse_ptrs, flag_ptrs, rank, epoch, timeout_us, status_ptr, B, H,
+                          Lq, q0, q1, out_ptr, lse_out_ptr=None, stream=0) -> None:
+    """nvkv_lse_merge behind the bounded cross-rank flag barrier; flag_ptrs:
+    device addresses (ints) of every rank's signal array."""
+    n = len(o_ptrs)
+    if len(lse_ptrs) != n or len(flag_ptrs) != n:
+        raise ValueError("one lse and one flag array per part")
+    oa = (ctypes.c_void_p * max(n, 1))(*o_ptrs)
+    la = (ctypes.c_void_p * max(n, 1))(*lse_ptrs)
+    fa = (ctypes.c_void_p * max(n, 1))(*flag_ptrs)
+    _check(lib.nvkv_lse_merge_synced(n, oa, la, fa, rank, epoch, timeout_us, status_ptr, B, H, Lq,
+                                     q0, q1, out_ptr, lse_out_ptr, stream),
+           "nvkv_lse_merge_synced")
 
 
 NVKV_FAULT_NONE = 0

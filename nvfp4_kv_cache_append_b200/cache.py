@@ -73,6 +73,11 @@ class KVCache:
         return self.T // self.desc.shard_count
 
     @property
+    def Tr(self) -> int:
+        """Rows of each frame slot: Ts, plus one padding row when Ts is odd."""
+        return (self.Ts + 1) // 2 * 2
+
+    @property
     def tok_off(self) -> int:
         """Index within the frame of the first cached token."""
         return self.desc.shard_rank * self.Ts
@@ -83,7 +88,7 @@ class KVCache:
 
     @property
     def rows(self) -> int:
-        return (self.desc.S + self.desc.W) * self.Ts
+        return (self.desc.S + self.desc.W) * self.Tr
 
     def footprint_bytes(self) -> int:
         ts = [self.k_data, self.v_data, self.k_scales, self.v_scales, self.amax, self.s_g,

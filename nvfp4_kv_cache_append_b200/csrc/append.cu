@@ -114,7 +114,9 @@ __device__ __forceinline__ float head_scale(const AppendLaunch &a, int gi, bool 
 // of the token-head: 64 bytes in, 16 code bytes and 2 scale bytes out),
 // threadIdx.y = token in the CTA's token group.  grid = (ceil(C Ts / ty), 2B):
 // blockIdx.y = t * B + b with t = 0 for K and 1 for V.  Row l of the grid is
-// token tok_off + l % Ts of chunk frame l / Ts (all tokens: Ts = T).
+// token tok_off + l % Ts of chunk frame l / Ts (all tokens: Ts = T), stored
+// in row l % Ts of its frame's slot (Tr rows per slot; the padding row of an
+// odd Ts is never written).
 __global__ void __launch_bounds__(512) k_nvfp4_append(const __grid_constant__ AppendLaunch a)
 {
     const int t = blockIdx.y / a.B, b = blockIdx.y - t * a.B;
@@ -130,7 +132,7 @@ __global__ void __launch_bounds__(512) k_nvfp4_append(const __grid_constant__ Ap
     const int gi = (t * a.B + b) * a.H + h;
     const float sg = head_scale(a, gi, l == 0 && pr == 0);
     const int slot = a.slot[b * a.C + frame];
-    quantize_pair(a, t, h, pr, (size_t)(b * a.H + h) * a.R + (size_t)slot * a.Ts + tok, sg, w0, w1,
+    quantize_pair(a, t, h, pr, (size_t)(b * a.H + h) * a.R + (size_t)slot * a.Tr + tok, sg, w0, w1,
                   w2, w3);
 }
 
@@ -146,7 +148,7 @@ __global__ void __launch_bounds__(1024) k_bf16_append(const __grid_constant__ Ap
     const uint4 *src = reinterpret_cast<const uint4 *>(t ? a.v : a.k) +
                        (((size_t)b * a.Lq + frame * a.T + a.tok_off + tok) * a.H + h) * 16 + c;
     const int slot = a.slot[b * a.C + frame];
-    const size_t row = (size_t)(b * a.H + h) * a.R + (size_t)slot * a.Ts + tok;
+    const size_t row = (size_t)(b * a.H + h) * a.R + (size_t)slot * a.Tr + tok;
     reinterpret_cast<uint4 *>(t ? a.v_data : a.k_data)[row * 16 + c] = ld_stream(src);
 }
 

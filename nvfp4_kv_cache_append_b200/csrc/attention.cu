@@ -111,6 +111,7 @@ struct SharedCtl {
     uint32_t tmem_base;
     int n_seg;
     int merge_flag;
+    float qinv[BM];     // per query row of the segment: 2^-e of its Q range scaling
     Segment seg[MAX_SEG];
 };
 
@@ -270,7 +271,7 @@ __device__ __forceinline__ bool wait_warp(Ctx &c, int bar, uint32_t parity)
 
 __device__ __forceinline__ int key_tiles(const AttnLaunch &a, int b)
 {
-    return (a.n_vis[b] * a.Tk + BN - 1) / BN;
+    return (a.n_vis[b] * a.Tr + BN - 1) / BN;
 }
 
 __device__ __forceinline__ long long total_tiles(const AttnLaunch &a)
@@ -389,31 +390,47 @@ struct KeyPos {
     size_t grow;   // global row index into the [B][H][R] planes
 };
 
+// Keys are numbered Tr per visible frame: key f Tr + i is row i of frame f's
+// slot, a token for i < Tk and the padding row (invalid) for i = Tk.
 // tok_off: index within the frame of the cache's first token (a shard of a
-// sequence-parallel KV split), a constant 0 for a whole cache
+// sequence-parallel KV split), a constant 0 for a whole cache.
 __device__ __forceinline__ KeyPos key_pos(const Ctx &c, int b, int h, int n_keys, int key,
                                           int tok_off)
 {
     const AttnLaunch &a = *c.a;
     KeyPos k;
-    k.valid = key < n_keys;
-    const int kk = k.valid ? key : 0;
-    const int f = div_fast(kk, a.Tk, a.inv_Tk);
-    const int tok = kk - f * a.Tk;
+    const int kk = key < n_keys ? key : 0;
+    const int f = div_fast(kk, a.Tr, a.inv_Tr);
+    const int tok = kk - f * a.Tr;
+    k.valid = key < n_keys && tok < a.Tk;
     const VisFrame vf = a.vis[b][f];
-    const int ft = tok_off + tok;             // the token's index in its frame
+    const int ft = tok_off + min(tok, a.Tk - 1);   // the token's index in its frame
     const int hp = div_fast(ft, a.grid_w, a.inv_grid_w);
     k.rr = rope_rows(c, vf.rope_pos, hp, ft - hp * a.grid_w);
-    k.grow = (size_t)(b * a.H + h) * a.R + (size_t)vf.slot * a.Tk + tok;
+    k.grow = (size_t)(b * a.H + h) * a.R + (size_t)vf.slot * a.Tr + tok;
     return k;
+}
+
+// 0 for the padding key of an odd shard (key mod Tr == Tk), else 1
+__device__ __forceinline__ bool not_pad(const AttnLaunch &a, int key)
+{
+    const int f = div_fast(key, a.Tr, a.inv_Tr);
+    return key - f * a.Tr < a.Tk;
 }
 
 // ------------------------------------------------------------ Q prologue
 
-// Q row `row` of the chunk -> RoPE in f32 -> f16 pairs in TMEM columns
-// [tcol, tcol + 64) of this thread's lane.
+// Q row `row` of the chunk -> times 2^e -> RoPE in f32 -> f16 pairs in TMEM
+// columns [tcol, tcol + 64) of this thread's lane; 2^-e is returned in
+// qinv_out.  e puts the row's largest |q| in [2^13, 2^14), so that the
+// rotated row (|rot| <= sqrt(2) max |q|) lies inside f16's normal range for
+// any finite bf16 input; the softmax multiplies its logit scale by 2^-e.  A
+// power of two commutes exactly with the f16 rounding (normal range), the
+// products and the f32 sums of S = Q K^T, so for rows already inside the
+// range the logits are unchanged bit for bit.  The row is read twice (its
+// max, then the values), the second time from L1.
 template <bool FP4>
-__device__ void load_q_tmem(const Ctx &c, int b, int h, int row, uint32_t tcol)
+__device__ void load_q_tmem(const Ctx &c, int b, int h, int row, uint32_t tcol, float &qinv_out)
 {
     const AttnLaunch &a = *c.a;
     const bool valid = row < a.Lq;
@@ -423,26 +440,43 @@ __device__ void load_q_tmem(const Ctx &c, int b, int h, int row, uint32_t tcol)
     const int tok = valid ? row - frame * a.T : 0;
     const int hp = div_fast(tok, a.grid_w, a.inv_grid_w);
     const RopeRows rr = rope_rows(c, a.q_pos0[b] + frame, hp, tok - hp * a.grid_w);
+    uint32_t mx = 0;                           // max |bf16| bits, both halves
+    if (valid) {
+#pragma unroll 1
+        for (int ch = 0; ch < 16; ++ch) {
+            const uint4 w = ldg16(src + ch);
+            mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu),
+                                       __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu)));
+        }
+    }
+    mx = max(mx >> 16, mx & 0xFFFFu);          // bf16 bits of max |q|
+    // e = 13 - floor(log2 max |q|), from the biased exponent; 0 for a zero row
+    // (or one holding infinities or NaN); kept inside [-126, 126]
+    const int ebits = (int)((mx >> 7) & 0xFFu);
+    int e = (mx == 0 || ebits == 0xFF) ? 0 : 140 - ebits;
+    e = max(-126, min(126, e));
+    const float up = __uint_as_float((uint32_t)(127 + e) << 23);
+    qinv_out = __uint_as_float((uint32_t)(127 - e) << 23);
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
         uint32_t o[32];
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
-            const uint4 w = valid ? ldg16(src + hh * 8 + ch) : make_uint4(0, 0, 0, 0);
-            const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+            const uint4 wv = valid ? ldg16(src + hh * 8 + ch) : make_uint4(0, 0, 0, 0);
+            const uint32_t u[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int p = hh * 32 + ch * 4 + k;
-                const float x = __uint_as_float(u[k] << 16);
-                const float y = __uint_as_float(u[k] & 0xFFFF0000u);
-                const uint2 e = lds8(rope_at(rr, p));
+                const float x = __uint_as_float(u[k] << 16) * up;
+                const float y = __uint_as_float(u[k] & 0xFFFF0000u) * up;
+                const uint2 e2 = lds8(rope_at(rr, p));
                 float cs, sn;
                 if (FP4) {
-                    cs = __low2float(as_h2(e.x));
-                    sn = __high2float(as_h2(e.y));
+                    cs = __low2float(as_h2(e2.x));
+                    sn = __high2float(as_h2(e2.y));
                 } else {
-                    cs = __uint_as_float(e.x);
-                    sn = __uint_as_float(e.y);
+                    cs = __uint_as_float(e2.x);
+                    sn = __uint_as_float(e2.y);
                 }
                 o[ch * 4 + k] = pack_f16(x * cs - y * sn, x * sn + y * cs);
             }
@@ -559,10 +593,13 @@ __device__ void k_converter_role(Ctx &c)
     int g = 0;                                 // tiles processed by this CTA
     for (int si = 0; si < c.ctl->n_seg; ++si) {
         const Segment sg = c.ctl->seg[si];
-        const int n_keys = a.n_vis[sg.b] * a.Tk;
+        const int n_keys = a.n_vis[sg.b] * a.Tr;
         if (si > 0 && !wait_warp(c, B_QFREE, (si - 1) & 1)) return;
         ptx::tc_fence_after();
-        load_q_tmem<FP4>(c, sg.b, sg.h, (2 * sg.p + (int)c.rank) * BM + t, tmem + lane_off + TM_Q);
+        float qi;
+        load_q_tmem<FP4>(c, sg.b, sg.h, (2 * sg.p + (int)c.rank) * BM + t,
+                         tmem + lane_off + TM_Q, qi);
+        c.ctl->qinv[t] = qi;                  // published by the QREADY arrive
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         arrive_x(c, B_QREADY);
@@ -597,7 +634,7 @@ __device__ void v_converter_role(Ctx &c)
     int g = 0;
     for (int si = 0; si < c.ctl->n_seg; ++si) {
         const Segment sg = c.ctl->seg[si];
-        const int n_keys = a.n_vis[sg.b] * a.Tk;
+        const int n_keys = a.n_vis[sg.b] * a.Tr;
         for (int tile = sg.t0; tile < sg.t1; ++tile, ++g) {
             const int s = g % NSTAGE, vb = g & 1;
             const uint32_t stg = c.sbase + OFF_STG + s * STG_BYTES;
@@ -605,7 +642,8 @@ __device__ void v_converter_role(Ctx &c)
             if (FP4 && !wait(c, B_STG_FULL + s, (g / NSTAGE) & 1)) return;
             if (g >= 2 && !wait(c, B_VFREE + vb, ((g - 2) >> 1) & 1)) return;
             if (FP4) {
-                conv_v_fp4(stg, k, (int)c.rank, tile * BN + k < n_keys, vdst);
+                conv_v_fp4(stg, k, (int)c.rank,
+                           tile * BN + k < n_keys && (!SHARD || not_pad(a, tile * BN + k)), vdst);
             } else {
                 const KeyPos kp = key_pos(c, sg.b, sg.h, n_keys, tile * BN + k, SHARD ? a.tok_off : 0);
                 conv_v_bf16(c, k, (int)c.rank, kp, vdst);
@@ -664,7 +702,7 @@ __device__ void relay_p_role(Ctx &c)
 
 // Bulk copies of one tile's packed rows: this CTA's 64 K rows and all 128 V
 // rows.  Every run of consecutive keys inside one frame is contiguous in the
-// planes; run starts and lengths are even (T even), so every copy is 16-byte
+// planes; run starts and lengths are even (Tr even, tiles of 64 keys), so every copy is 16-byte
 // aligned and sized.
 __device__ __forceinline__ void copy_runs(const AttnLaunch &a, int b, size_t head_row0, int k0,
                                           int k1, uint8_t *dst_c, uint8_t *dst_s,
@@ -672,9 +710,9 @@ __device__ __forceinline__ void copy_runs(const AttnLaunch &a, int b, size_t hea
                                           uint64_t *full)
 {
     for (int k = k0; k < k1;) {
-        const int f = div_fast(k, a.Tk, a.inv_Tk), tok = k - f * a.Tk;
-        const int n = min(a.Tk - tok, k1 - k);
-        const size_t g = head_row0 + (size_t)a.vis[b][f].slot * a.Tk + tok;
+        const int f = div_fast(k, a.Tr, a.inv_Tr), tok = k - f * a.Tr;
+        const int n = min(a.Tr - tok, k1 - k);
+        const size_t g = head_row0 + (size_t)a.vis[b][f].slot * a.Tr + tok;
         const int t0 = k - k0;
         ptx::bulk_g2s(dst_c + t0 * 64, codes + g * 64, (uint32_t)n * 64, full);
         ptx::bulk_g2s(dst_s + t0 * 8, scales + g * 8, (uint32_t)n * 8, full);
@@ -692,7 +730,7 @@ __device__ void producer_role(Ctx &c)
     bool ok = true;
     for (int si = 0; ok && si < c.ctl->n_seg; ++si) {
         const Segment sg = c.ctl->seg[si];
-        const int n_keys = a.n_vis[sg.b] * a.Tk;
+        const int n_keys = a.n_vis[sg.b] * a.Tr;
         const size_t head_row0 = (size_t)(sg.b * a.H + sg.h) * a.R;
         for (int tile = sg.t0; tile < sg.t1; ++tile, ++g) {
             const int s = g % NSTAGE;
@@ -827,7 +865,7 @@ __device__ __forceinline__ void store_row_bf16(uint4 *dst, const float *acc, flo
     }
 }
 
-template <bool FP4>
+template <bool FP4, bool SHARD>
 __device__ void softmax_role(Ctx &c)
 {
     const AttnLaunch &a = *c.a;
@@ -841,11 +879,19 @@ __device__ void softmax_role(Ctx &c)
     int g = 0;
     for (int si = 0; si < c.ctl->n_seg; ++si) {
         const Segment sg = c.ctl->seg[si];
-        const int n_keys = a.n_vis[sg.b] * a.Tk;
+        const int n_keys = a.n_vis[sg.b] * a.Tr;
         const int gi = sg.b * a.H + sg.h;
         const float sgk = FP4 ? a.s_g[gi] : 1.0f;
         const float sgv = FP4 ? a.s_g[a.B * a.H + gi] : 1.0f;
-        const float scale = sgk * 1.4426950408889634f * 0.08838834764831845f;   // log2(e)/sqrt(128)
+        // this row's Q range scaling, written with the segment's Q tile:
+        // wait for that tile (its phase cannot run ahead: the next segment's
+        // Q waits for this segment's last PV, which needs this thread's P)
+        if (!wait_warp(c, B_QREADY, si & 1)) return;
+        ptx::tc_fence_after();
+        const float qinv = c.ctl->qinv[r];
+        // log2(e)/sqrt(128) times s_g(K) times the row's 2^-e (all exact
+        // powers of two but the first)
+        const float scale = sgk * 1.4426950408889634f * 0.08838834764831845f * qinv;
         float m = -INFINITY, l = 0.0f;
         for (int tile = sg.t0; tile < sg.t1; ++tile, ++g) {
             const int buf = g & 1;
@@ -869,6 +915,17 @@ __device__ void softmax_role(Ctx &c)
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
                         if (q * 32 + i >= nv) s[i] = -INFINITY;
+                }
+                if (SHARD && a.Tr != a.Tk) {
+                    // padding keys (one per frame, key mod Tr == Tk) of this chunk
+                    const int k0 = tile * BN + q * 32;
+                    uint32_t pad = 0;
+                    for (int i = a.Tk - (k0 - div_fast(k0, a.Tr, a.inv_Tr) * a.Tr); i < 32;
+                         i += a.Tr)
+                        if (i >= 0) pad |= 1u << i;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if ((pad >> i) & 1u) s[i] = -INFINITY;
                 }
                 float mx4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
@@ -1013,8 +1070,9 @@ __device__ void softmax_role(Ctx &c)
 
 // ------------------------------------------------------------ kernel
 
-// VAR 0: a whole cache; 1 (SHARD): a shard whose first token is not token 0
-// of the frame; 2: the failure-path test.  Separate instantiations keep the
+// VAR 0: a whole cache with an even number of tokens per frame; 1 (SHARD):
+// a shard whose first token is not token 0 of the frame, or whose slots hold
+// a padding row (odd token count); 2: the failure-path test.  Separate instantiations keep the
 // whole-cache kernel's code free of both.
 template <bool FP4, int VAR>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
@@ -1064,7 +1122,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     ptx::tc_fence_after();
 
     if (warp < 4) {
-        softmax_role<FP4>(c);
+        softmax_role<FP4, VAR == 1>(c);
     } else if (warp < 8) {
         k_converter_role<FP4, VAR == 1>(c);
     } else if (warp < 12) {
@@ -1130,7 +1188,7 @@ cudaError_t launch_chunk_attention(const AttnLaunch &a, cudaStream_t s)
 {
     const bool fp4 = a.kv_dtype == NVKV_KV_NVFP4;
     if (fp4 && a.fault == NVKV_FAULT_SKIP_FIRST_STAGE && !a.tok_off) return launch<true, 2>(a, s);
-    if (a.tok_off) return fp4 ? launch<true, 1>(a, s) : launch<false, 1>(a, s);
+    if (a.tok_off || a.Tr != a.Tk) return fp4 ? launch<true, 1>(a, s) : launch<false, 1>(a, s);
     return fp4 ? launch<true, 0>(a, s) : launch<false, 0>(a, s);
 }
 

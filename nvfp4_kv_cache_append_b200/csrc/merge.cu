@@ -14,6 +14,16 @@
 // chunk of every part's bf16 row), so a warp reads two whole 256-byte rows of
 // each part.  HBM-bound: n * (256 + 4) bytes read and 256 (+ 4) written per
 // row.
+//
+// The synced form puts the step's cross-rank barrier in the same kernel: each
+// CTA first signals every rank that this rank's part is complete (a store
+// with release semantics at system scope into that rank's flag array; the
+// part was written by earlier work on this stream), then waits for the
+// signals of all ranks (acquire loads, bounded in time) before it reads
+// their parts.  Any CTA that runs signals, so the barrier cannot deadlock
+// on CTAs not yet resident; repeated signals store the same value.  A wait
+// that runs out records NVKV_ERR_TIMEOUT in the status word and the CTA
+// returns without reading (no trap, the context stays usable).
 #include <cuda_bf16.h>
 
 #include "nvkv_internal.h"
@@ -33,8 +43,57 @@ __device__ __forceinline__ uint4 ld_part(const void *base, size_t idx)
     return r;
 }
 
+__device__ __forceinline__ void st_release_sys(uint32_t *p, uint32_t v)
+{
+    asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_sys(const uint32_t *p)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint64_t now_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// signal every rank, then wait for every rank's signal of this epoch; false
+// (block-uniform) if a wait ran out or another CTA already reported an error
+__device__ bool cross_rank_barrier(const MergeLaunch &m)
+{
+    const int j = threadIdx.x;
+    if (j < m.n) st_release_sys(m.flags[j] + m.rank, m.epoch);
+    bool ok = true;
+    if (j < m.n && j != m.rank) {
+        const uint32_t *f = m.flags[m.rank] + j;
+        const volatile int32_t *st = m.status;
+        const uint64_t t0 = now_ns();
+        // wrap-safe: the flag has reached epoch once (flag - epoch) is
+        // non-negative as a signed difference
+        while ((int32_t)(ld_acquire_sys(f) - m.epoch) < 0) {
+            if (*st != 0) {
+                ok = false;
+                break;
+            }
+            if (now_ns() - t0 > m.timeout_ns) {
+                atomicCAS(m.status, 0, (int32_t)NVKV_ERR_TIMEOUT);
+                ok = false;
+                break;
+            }
+            __nanosleep(256);
+        }
+    }
+    return __syncthreads_and(ok) != 0;
+}
+
 __global__ void __launch_bounds__(kThreads) k_lse_merge(const __grid_constant__ MergeLaunch m)
 {
+    if (m.sync && !cross_rank_barrier(m)) return;
     const long long rows = (long long)m.B * m.nq * m.H;
     const long long r = (long long)blockIdx.x * (kThreads / 16) + (threadIdx.x >> 4);
     if (r >= rows) return;

@@ -50,7 +50,7 @@ nvkv_status check_desc(const nvkv_desc *d)
     if (d->shard_count < 1 || d->shard_count > NVKV_MAX_SHARDS || d->shard_rank < 0 ||
         d->shard_rank >= d->shard_count || T % d->shard_count)
         return NVKV_ERR_INVALID_ARG;
-    const int64_t R = T / d->shard_count * (d->S + d->W);
+    const int64_t R = (T / d->shard_count + 1) / 2 * 2 * (d->S + d->W);
     // 32-bit index arithmetic in the kernels
     if (R * d->B * d->H * 128 >= (int64_t(1) << 31) / 2 ||
         T * d->C * d->B * d->H * 128 >= (int64_t(1) << 31) / 2)
@@ -69,7 +69,7 @@ nvkv_status check_ring(const nvkv_desc *d, const nvkv_ring *r)
     return NVKV_OK;
 }
 
-int64_t rows_per_head(const nvkv_desc *d) { return (int64_t)nvkv::shard_tokens(d) * (d->S + d->W); }
+int64_t rows_per_head(const nvkv_desc *d) { return (int64_t)nvkv::slot_rows(d) * (d->S + d->W); }
 
 bool is_visible(const nvkv_ring_stream &s, int i)
 {
@@ -177,6 +177,7 @@ nvkv_status append_common(const nvkv_desc *desc, const nvkv_cache *cache, const 
     a.Lq = desc->C * a.T;
     a.Ts = nvkv::shard_tokens(desc);
     a.tok_off = nvkv::shard_first_token(desc);
+    a.Tr = nvkv::slot_rows(desc);
     a.R = (int)rows_per_head(desc);
     a.C = desc->C;
     a.first = overwrite ? (ring->steps == 1 ? 1 : 0) : (ring->scales_fixed ? 0 : 1);
@@ -246,12 +247,13 @@ nvkv_status attention_common(const nvkv_desc *desc, const nvkv_cache *cache,
     a.inv_grid_w = 1.0f / (float)desc->grid_w;
     a.Tk = nvkv::shard_tokens(desc);
     a.tok_off = nvkv::shard_first_token(desc);
-    a.inv_Tk = 1.0f / (float)a.Tk;
-    // the attention kernels are built for the 44/42/42 split and small grids;
-    // the NVFP4 kernel stages scale rows with 16-byte bulk copies, which needs
-    // an even number of cached tokens per frame
+    // keys are numbered Tr per frame, the padding row of an odd Tk included
+    // (masked), so that every run of rows the kernel copies is 16-byte sized
+    a.Tr = nvkv::slot_rows(desc);
+    a.inv_Tr = 1.0f / (float)a.Tr;
+    // the attention kernels are built for the 44/42/42 split and small grids
     if (desc->rope_split[0] != 44 || desc->rope_split[1] != 42 || desc->rope_split[2] != 42 ||
-        desc->grid_h > 256 || desc->grid_w > 256 || (dtype == NVKV_KV_NVFP4 && (a.Tk & 1)))
+        desc->grid_h > 256 || desc->grid_w > 256)
         return NVKV_ERR_UNSUPPORTED;
     {
         int p = 0;
@@ -283,7 +285,7 @@ nvkv_status attention_common(const nvkv_desc *desc, const nvkv_cache *cache,
     a.n_pairs = query_pairs(desc);
     int64_t total = 0, min_tiles = INT64_MAX;
     for (int b = 0; b < desc->B; ++b) {
-        const int64_t nkt = ceil_div((int64_t)a.n_vis[b] * a.Tk, kTileKeys);
+        const int64_t nkt = ceil_div((int64_t)a.n_vis[b] * a.Tr, kTileKeys);
         total += (int64_t)desc->H * a.n_pairs * nkt;
         min_tiles = std::min(min_tiles, nkt);
     }
@@ -341,7 +343,6 @@ nvkv_status nvkv_desc_set_shard(nvkv_desc *desc, int rank, int count)
     d.shard_count = count;
     nvkv_status st = check_desc(&d);
     if (st != NVKV_OK) return st;
-    if (d.kv_dtype == NVKV_KV_NVFP4 && (nvkv::shard_tokens(&d) & 1)) return NVKV_ERR_UNSUPPORTED;
     *desc = d;
     return NVKV_OK;
 }
@@ -493,8 +494,8 @@ size_t nvkv_attention_workspace_bytes(const nvkv_desc *desc)
     const int dev_slots = nvkv::attention_slots(dev);
     if (dev_slots < 1) return 0;
     // bound over every ring state: at most S + W visible frames, at least the
-    // chunk's own C frames
-    const int64_t T = nvkv::shard_tokens(desc);
+    // chunk's own C frames (keys are numbered slot_rows per frame)
+    const int64_t T = nvkv::slot_rows(desc);
     const int64_t max_tiles = ceil_div((desc->S + desc->W) * T, kTileKeys);
     const int64_t min_tiles = ceil_div(desc->C * T, kTileKeys);
     const int64_t total = (int64_t)desc->B * desc->H * query_pairs(desc) * max_tiles;
@@ -542,6 +543,7 @@ nvkv::ProjLaunch project_launch(const nvkv_desc *desc, int hidden)
     p.M = desc->B * p.Lq;
     p.hidden = hidden;
     p.R = (int)rows_per_head(desc);
+    p.Tr = nvkv::slot_rows(desc);
     return p;
 }
 
@@ -613,15 +615,17 @@ nvkv_status nvfp4_kv_project_append(const nvkv_desc *desc, const nvkv_cache *cac
     return NVKV_OK;
 }
 
-nvkv_status nvkv_lse_merge(int n_parts, const void *const *o_parts, const float *const *lse_parts,
-                           int B, int H, int Lq, int q0, int q1, void *out, float *lse_out,
-                           nvkv_stream stream)
+namespace {
+
+nvkv_status merge_setup(int n_parts, const void *const *o_parts, const float *const *lse_parts,
+                        int B, int H, int Lq, int q0, int q1, void *out, float *lse_out,
+                        nvkv::MergeLaunch &m)
 {
     if (n_parts < 1 || n_parts > NVKV_MAX_SHARDS || !o_parts || !lse_parts || !out || B < 1 ||
         H < 1 || Lq < 1 || q0 < 0 || q1 > Lq || q0 >= q1)
         return NVKV_ERR_INVALID_ARG;
     if ((int64_t)B * Lq * H * 128 >= (int64_t(1) << 31)) return NVKV_ERR_UNSUPPORTED;
-    nvkv::MergeLaunch m{};
+    m = nvkv::MergeLaunch{};
     for (int j = 0; j < n_parts; ++j) {
         if (!o_parts[j] || !lse_parts[j]) return NVKV_ERR_INVALID_ARG;
         if (!aligned16(o_parts[j]) || (reinterpret_cast<uintptr_t>(lse_parts[j]) & 3u))
@@ -638,6 +642,43 @@ nvkv_status nvkv_lse_merge(int n_parts, const void *const *o_parts, const float 
     m.nq = q1 - q0;
     m.out = out;
     m.lse_out = lse_out;
+    return NVKV_OK;
+}
+
+}  // namespace
+
+nvkv_status nvkv_lse_merge(int n_parts, const void *const *o_parts, const float *const *lse_parts,
+                           int B, int H, int Lq, int q0, int q1, void *out, float *lse_out,
+                           nvkv_stream stream)
+{
+    nvkv::MergeLaunch m;
+    const nvkv_status st = merge_setup(n_parts, o_parts, lse_parts, B, H, Lq, q0, q1, out, lse_out, m);
+    if (st != NVKV_OK) return st;
+    return nvkv::launch_lse_merge(m, (cudaStream_t)stream) == cudaSuccess ? NVKV_OK : NVKV_ERR_CUDA;
+}
+
+nvkv_status nvkv_lse_merge_synced(int n_parts, const void *const *o_parts,
+                                  const float *const *lse_parts, uint32_t *const *flags, int rank,
+                                  uint32_t epoch, uint32_t timeout_us, int32_t *status, int B,
+                                  int H, int Lq, int q0, int q1, void *out, float *lse_out,
+                                  nvkv_stream stream)
+{
+    nvkv::MergeLaunch m;
+    const nvkv_status st = merge_setup(n_parts, o_parts, lse_parts, B, H, Lq, q0, q1, out, lse_out, m);
+    if (st != NVKV_OK) return st;
+    if (!flags || !status || rank < 0 || rank >= n_parts || epoch == 0 || timeout_us == 0)
+        return NVKV_ERR_INVALID_ARG;
+    for (int j = 0; j < n_parts; ++j) {
+        if (!flags[j]) return NVKV_ERR_INVALID_ARG;
+        if (reinterpret_cast<uintptr_t>(flags[j]) & 3u) return NVKV_ERR_ALIGNMENT;
+        m.flags[j] = flags[j];
+    }
+    if (reinterpret_cast<uintptr_t>(status) & 3u) return NVKV_ERR_ALIGNMENT;
+    m.sync = 1;
+    m.rank = rank;
+    m.epoch = epoch;
+    m.timeout_ns = (uint64_t)timeout_us * 1000u;
+    m.status = status;
     return nvkv::launch_lse_merge(m, (cudaStream_t)stream) == cudaSuccess ? NVKV_OK : NVKV_ERR_CUDA;
 }
 

@@ -18,6 +18,7 @@ struct AppendLaunch {
     float *s_g;                      // [2][B][H]
     int B, H, T, Lq, R, C;           // T tokens per frame, Lq = C * T rows of k, v
     int Ts, tok_off;                 // this shard's tokens of a frame: [tok_off, tok_off + Ts)
+    int Tr;                          // rows per frame slot (Ts rounded up to even)
     float inv_Ts;                    // 1/Ts, set by the launchers (frame index by reciprocal)
     int first;                       // 1: measure amax and fix s_g
     int32_t slot[NVKV_MAX_BATCH * NVKV_MAX_CHUNK];  // [b * C + c] -> physical slot
@@ -30,6 +31,10 @@ inline int shard_tokens(const nvkv_desc *d)
     return d->grid_h * d->grid_w / (d->shard_count > 0 ? d->shard_count : 1);
 }
 inline int shard_first_token(const nvkv_desc *d) { return d->shard_rank * shard_tokens(d); }
+// Rows of a frame slot: the shard's tokens, plus one padding row when their
+// count is odd, so that every slot starts on a 16-byte boundary of the
+// 8-byte-per-row scale planes.
+inline int slot_rows(const nvkv_desc *d) { return (shard_tokens(d) + 1) & ~1; }
 
 cudaError_t launch_nvfp4_append(const AppendLaunch &a, cudaStream_t s);
 // nvfp4_kv_append with its amax scratch given by the caller (amax_scratch
@@ -65,7 +70,8 @@ struct AttnLaunch {
     int grid_h;
     float inv_T, inv_grid_w;         // 1/T and 1/grid_w (division by reciprocal + fix-up)
     int Tk, tok_off;                 // cached tokens per frame (the shard's), first one's index
-    float inv_Tk;                    // 1/Tk
+    int Tr;                          // rows per frame slot: Tk, or Tk + 1 (one padding row)
+    float inv_Tr;                    // 1/Tr
     int n_fpos;                      // frame positions used: 0 .. n_fpos-1
     float theta[64];                 // RoPE angle per unit position of each channel pair
     void *workspace;                 // split-item partials + counters (zero on first use)
@@ -87,6 +93,7 @@ cudaError_t launch_chunk_attention(const AttnLaunch &a, cudaStream_t s);
 struct ProjLaunch {
     int M, hidden;                   // rows of x (B * Lq), hidden (multiple of 64)
     int B, H, Lq, T, R, C;
+    int Tr;                          // rows per frame slot
     int mode;
     void *k_out, *v_out;             // mode 0: bf16 [B][Lq][H][128]
     void *k_data, *v_data;           // mode 1: NVFP4 planes of the cache
@@ -107,6 +114,14 @@ struct MergeLaunch {
     int n, B, H, Lq, q0, nq;
     void *out;                          // bf16 [B][nq][H][128]
     float *lse_out;                     // f32 [B][H][nq] or null
+    // cross-rank barrier fused in front of the merge (sync = 1): rank `rank`
+    // stores `epoch` into flags[j][rank] of every part j, then waits until
+    // flags[rank][j] reaches epoch for every j, at most timeout_ns
+    int sync, rank;
+    uint32_t epoch;
+    uint32_t *flags[NVKV_MAX_SHARDS];
+    uint64_t timeout_ns;
+    int32_t *status;
 };
 
 cudaError_t launch_lse_merge(const MergeLaunch &m, cudaStream_t s);

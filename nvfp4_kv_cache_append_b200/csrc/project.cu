@@ -240,7 +240,7 @@ __device__ void epilogue(PCtx &c)
             size_t drow = 0;
             float sg = 1.0f;
             if (p.mode == 1) {
-                drow = (size_t)(bi * p.H + h) * p.R + (size_t)p.slot[bi * p.C + frame] * p.T + tok;
+                drow = (size_t)(bi * p.H + h) * p.R + (size_t)p.slot[bi * p.C + frame] * p.Tr + tok;
                 sg = p.s_g[(kv * p.B + bi) * p.H + h];
             }
 #pragma unroll 1

@@ -12,17 +12,21 @@ step on every rank:
   2. attention of the whole chunk's queries over the shard's keys, with the
      lse, into this rank's half of a double-buffered partial-result buffer in
      symmetric memory (every rank can load every other rank's buffer);
-  3. one cross-rank barrier on the stream;
-  4. ``nvkv_lse_merge`` of query rows [r*Lq/n, (r+1)*Lq/n) (this rank's
-     slice of the chunk) reading all n partial results, n - 1 of them from
-     the peers' memory over NVLink: the exchange and the merge are one kernel.
+  3. ``nvkv_lse_merge_synced``: one kernel that signals every rank through
+     device flags in the same symmetric buffer, waits (bounded) for every
+     rank's signal of this step, then merges query rows [r*Lq/n, (r+1)*Lq/n)
+     (this rank's slice of the chunk) from all n partial results, n - 1 of
+     them read from the peers' memory over NVLink: barrier, exchange and
+     merge are one launch.
 
 The rank ends the step with the attention output of its own query slice, the
 layout the rest of a sequence-parallel layer works on.  PyTorch provides the
-process group, the symmetric allocation and the barrier; the path runs in
-libnvkv.so's kernels.  The slot of the partial buffer alternates per step: a
-rank overwrites slot s only two steps later, after the barrier of the step in
-between, which every rank passes only once it has finished merging from s.
+process group and the symmetric allocation; the path runs in libnvkv.so's
+kernels.  A barrier wait that runs out writes NVKV_ERR_TIMEOUT to the cache's
+status word (``cache.device_status()``) instead of trapping.  The slot of the
+partial buffer alternates per step: a rank overwrites slot s only two steps
+later, after the barrier of the step in between, which every rank passes only
+once it has finished merging from s.
 """
 from __future__ import annotations
 
@@ -32,7 +36,7 @@ from typing import Optional, Tuple
 import torch
 
 from . import _lib as L
-from .cache import KVCache, lse_merge_ptrs
+from .cache import KVCache, _stream
 
 
 @dataclass(frozen=True)
@@ -63,6 +67,8 @@ class SequenceParallelKV:
     rank, NCCL); ``step`` returns the chunk attention of this rank's query
     slice over the whole cache."""
 
+    FLAG_BYTES = 64          # NVKV_MAX_SHARDS uint32 signals per rank
+
     def __init__(self, B: int, H: int, grid_h: int, grid_w: int, C: int, S: int, W: int,
                  kv_dtype: int = L.NVKV_KV_NVFP4, group=None, barrier_timeout_ms: int = 10000):
         import torch.distributed as dist
@@ -77,9 +83,15 @@ class SequenceParallelKV:
         self.o_bytes = B * self.Lq * H * 128 * 2
         self.l_bytes = B * H * self.Lq * 4
         self.slot_bytes = (self.o_bytes + self.l_bytes + 255) // 256 * 256
-        self.buf = symm_mem.empty(2 * self.slot_bytes, dtype=torch.uint8, device=device)
+        self.buf = symm_mem.empty(2 * self.slot_bytes + self.FLAG_BYTES, dtype=torch.uint8,
+                                  device=device)
         self.hdl = symm_mem.rendezvous(self.buf, self.group)
         self.ptrs = list(self.hdl.buffer_ptrs)
+        self.flag_ptrs = [p + 2 * self.slot_bytes for p in self.ptrs]
+        # every rank's flags are zero before any rank signals
+        self.buf[2 * self.slot_bytes:].zero_()
+        torch.cuda.synchronize(device)
+        dist.barrier(group=self.group)
         self.timeout_ms = barrier_timeout_ms
         self.steps = 0
 
@@ -97,11 +109,17 @@ class SequenceParallelKV:
         self.steps += 1
         o_part, l_part = self._slot_views(s)
         self.cache.step(q, k, v, out=o_part, lse=l_part)
-        self.hdl.barrier(channel=0, timeout_ms=self.timeout_ms)
         q0, q1 = self.plan.queries
         if out is None:
             out = torch.empty((self.B, q1 - q0, self.H, 128), dtype=torch.bfloat16, device=q.device)
+        elif tuple(out.shape) != (self.B, q1 - q0, self.H, 128) or out.dtype != torch.bfloat16 \
+                or not out.is_contiguous():
+            raise ValueError(f"out must be contiguous bf16 [{self.B}, {q1 - q0}, {self.H}, 128]")
         base = s * self.slot_bytes
-        return lse_merge_ptrs([p + base for p in self.ptrs],
-                              [p + base + self.o_bytes for p in self.ptrs],
-                              self.B, self.Lq, self.H, q0, q1, out)
+        epoch = self.steps & 0xFFFFFFFF or 1
+        L.nvkv_lse_merge_synced([p + base for p in self.ptrs],
+                                [p + base + self.o_bytes for p in self.ptrs], self.flag_ptrs,
+                                self.plan.rank, epoch, self.timeout_ms * 1000,
+                                self.cache.status.data_ptr(), self.B, self.H, self.Lq, q0, q1,
+                                out.data_ptr(), None, _stream(None))
+        return out

@@ -77,15 +77,21 @@ def test_shard_validation():
     assert (d.shard_rank, d.shard_count) == (3, 4)
     for rank, count, want in [(2, 2, "NVKV_ERR_INVALID_ARG"), (0, 0, "NVKV_ERR_INVALID_ARG"),
                               (0, 17, "NVKV_ERR_INVALID_ARG"), (-1, 2, "NVKV_ERR_INVALID_ARG"),
-                              (0, 7, "NVKV_ERR_INVALID_ARG"),      # 1560 tokens do not split in 7
-                              (0, 8, "NVKV_ERR_UNSUPPORTED")]:     # 195 tokens: odd for NVFP4
+                              (0, 7, "NVKV_ERR_INVALID_ARG")]:     # 1560 tokens do not split in 7
         e = nv.nvkv_desc_init(1, 12, 30, 52, 3, 3, 18)
         assert _status(nv.nvkv_desc_set_shard, e, rank, count) == want, (rank, count)
         assert (e.shard_rank, e.shard_count) == (0, 1)            # unchanged on error
-    t = nv.nvkv_desc_init(1, 12, 30, 52, 3, 3, 18, nv.NVKV_KV_BF16)
-    nv.nvkv_desc_set_shard(t, 7, 8)                                # the bf16 twin takes odd shares
-    nv.nvkv_desc_set_shard(t, 0, 1)
-    assert (t.shard_rank, t.shard_count) == (0, 1)
+    for kv in (nv.NVKV_KV_NVFP4, nv.NVKV_KV_BF16):
+        t = nv.nvkv_desc_init(1, 12, 30, 52, 3, 3, 18, kv)
+        nv.nvkv_desc_set_shard(t, 7, 8)                            # 195 tokens per shard (odd)
+        # 195 tokens + one padding row per slot, 21 slots, 12 heads
+        rows = 196 * 21 * 12
+        assert L.nvkv_plane_bytes(t, L.NVKV_PLANE_K_DATA) == rows * (64 if kv == 0 else 256)
+        if kv == nv.NVKV_KV_NVFP4:
+            assert L.nvkv_plane_bytes(t, L.NVKV_PLANE_K_SCALES) == rows * 8 + 16
+        nv.nvkv_desc_set_shard(t, 0, 1)
+        assert (t.shard_rank, t.shard_count) == (0, 1)
+        assert L.nvkv_plane_bytes(t, L.NVKV_PLANE_K_DATA) == 1560 * 21 * 12 * (64 if kv == 0 else 256)
 
 
 def test_merge_validation_before_launch():
@@ -103,6 +109,28 @@ def test_merge_validation_before_launch():
         la = (ctypes.c_void_p * max(n, 1))(*l)
         st = L.lib.nvkv_lse_merge(n, oa, la, *args[3:], None, None)
         assert L.STATUS[st] == want, (args, L.STATUS[st])
+
+
+def test_synced_merge_validation_before_launch():
+    fake = 1 << 20                                                 # never dereferenced
+    ok = dict(n=2, o=[fake, fake], l=[fake, fake], f=[fake, fake], rank=1, epoch=5, tmo=1000,
+              status=fake)
+    cases = [({}, None),
+             ({"rank": 2}, "NVKV_ERR_INVALID_ARG"), ({"rank": -1}, "NVKV_ERR_INVALID_ARG"),
+             ({"epoch": 0}, "NVKV_ERR_INVALID_ARG"), ({"tmo": 0}, "NVKV_ERR_INVALID_ARG"),
+             ({"status": None}, "NVKV_ERR_INVALID_ARG"), ({"f": [fake, 0]}, "NVKV_ERR_INVALID_ARG"),
+             ({"f": [fake, fake + 2]}, "NVKV_ERR_ALIGNMENT"), ({"status": fake + 1}, "NVKV_ERR_ALIGNMENT"),
+             ({"o": [fake, fake + 8]}, "NVKV_ERR_ALIGNMENT"), ({"n": 0}, "NVKV_ERR_INVALID_ARG")]
+    for change, want in cases:
+        if want is None:
+            continue                                               # a valid call would launch
+        a = dict(ok, **change)
+        n = a["n"]
+        arr = lambda v: (ctypes.c_void_p * 2)(*v)
+        st = L.lib.nvkv_lse_merge_synced(n, arr(a["o"]), arr(a["l"]), arr(a["f"]), a["rank"],
+                                         a["epoch"], a["tmo"], a["status"], 1, 2, 8, 0, 8, fake,
+                                         None, None)
+        assert L.STATUS[st] == want, (change, L.STATUS[st])
 
 
 def test_plane_bytes():

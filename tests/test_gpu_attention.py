@@ -112,3 +112,58 @@ def test_growing_logits_rescale(kv_dtype):
         for h in range(wl.H):
             ref, _ = ora.attention(0, h, np.arange(wl.Lq), quantized=quantized)
             assert_parity(got[0, :, h], ref, f"step {step} h {h}")
+
+
+def _scaled_run(wl, kv_dtype, qf, kf):
+    """Outputs and LSE of every step of `wl` with Q times qf and K times kf,
+    and the oracle's worst parity figures on every row."""
+    lib = LibStream(wl, kv_dtype)
+    ora = OracleStream(wl, seed=0, keep_inputs=True)
+    outs = []
+    for step in range(1, wl.steps + 1):
+        x = kvsynth.chunk_qkv(wl, step, 0)
+        q = (x["q"].float() * qf).to(torch.bfloat16)
+        k = (x["k"].float() * kf).to(torch.bfloat16)
+        ora.step(k=k, v=x["v"], q=q)
+        g = to_gpu({"q": q, "k": k, "v": x["v"]})
+        out, lse = lib.step(g["q"], g["k"], g["v"])
+        torch.cuda.synchronize()
+        assert lib.cache.device_status() == 0
+        got = out.float().cpu().numpy()
+        glse = lse.cpu().numpy()
+        for h in range(wl.H):
+            ref, ref_lse = ora.attention(0, h, np.arange(wl.Lq), quantized=kv_dtype == 0)
+            assert_parity(got[0, :, h], ref, f"q x {qf} k x {kf} step {step} h {h}")
+            assert np.abs(glse[0, h] - ref_lse).max() < 2e-2
+        outs.append((out.cpu(), lse.cpu()))
+    return outs
+
+
+# Q scaled by an exact power of two, K by its inverse: the logits are the same
+# real numbers (the NVFP4 quantization of K scales exactly with a power of
+# two: s_g moves, the codes and block scales do not), so the NVFP4 call must
+# return bit for bit what it returns on the unscaled inputs, and match the
+# oracle.  At 2^+-40 the rotated Q lies far outside f16 (overflow, or
+# subnormal loss) unless each row is range-scaled before the f16 rounding.
+@pytest.mark.parametrize("e", [12, -12, 40, -40])
+def test_q_range_compensated(e):
+    wl = kvsynth.WORKLOADS["tiny"]
+    base = _scaled_run(wl, 0, 1.0, 1.0)
+    got = _scaled_run(wl, 0, 2.0 ** e, 2.0 ** -e)
+    for (o0, l0), (o1, l1) in zip(base, got):
+        assert torch.equal(o0, o1)
+        assert torch.equal(l0, l1)
+
+
+# Q alone times 2^-12 (logits 4096 times smaller: near-uniform attention) on
+# both calls.  Q alone times 2^12 makes the softmax an argmax whose near-ties
+# are decided by the last bit of the rotated Q, so the compensated form above
+# stands in for it.
+@pytest.mark.parametrize("kv_dtype", [0, 1], ids=["nvfp4", "bf16"])
+def test_q_small(kv_dtype):
+    _scaled_run(kvsynth.WORKLOADS["tiny"], kv_dtype, 2.0 ** -12, 1.0)
+
+
+def test_q_large_bf16kv():
+    """The twin with Q times 2^12 and K times 2^-12 (K stays inside f16)."""
+    _scaled_run(kvsynth.WORKLOADS["tiny"], 1, 2.0 ** 12, 2.0 ** -12)

@@ -26,17 +26,28 @@ def _slot_of(cache, b, fid):
     raise KeyError(fid)
 
 
+# 60 tokens per frame in 4 shards: 15 per shard, an odd count, so every slot
+# carries a padding row; 25 tokens per frame: an odd whole cache
+ODD60 = kvsynth.Workload("odd60", B=2, H=3, D=128, grid_h=6, grid_w=10, C=2, S=1, W=6, steps=6)
+ODD25 = kvsynth.Workload("odd25", B=1, H=2, D=128, grid_h=5, grid_w=5, C=1, S=1, W=4, steps=7)
+
+
 @pytest.mark.parametrize("name,count,kv,steps", [
     ("tiny", 2, "nvfp4", 6), ("tiny", 4, "nvfp4", 6), ("tiny", 8, "bf16", 6),
-    ("stream5b", 2, "nvfp4", 4), ("stream5b", 4, "bf16", 3), ("stream1p3b", 4, "nvfp4", 3)])
+    ("stream5b", 2, "nvfp4", 4), ("stream5b", 4, "bf16", 3), ("stream1p3b", 4, "nvfp4", 3),
+    # 8 shards of the 1.3B-like stream: 195 tokens per shard (odd)
+    ("stream1p3b", 8, "nvfp4", 2),
+    (ODD60, 4, "nvfp4", 6), (ODD60, 4, "bf16", 4), (ODD25, 1, "nvfp4", 7)],
+    ids=lambda v: v.name if isinstance(v, kvsynth.Workload) else None)
 def test_shards_bit_exact_and_merge_to_whole_attention(name, count, kv, steps):
     import nvfp4_kv_cache_append_b200 as nv
-    wl = kvsynth.WORKLOADS[name]
+    wl = name if isinstance(name, kvsynth.Workload) else kvsynth.WORKLOADS[name]
     dtype = nv.NVKV_KV_NVFP4 if kv == "nvfp4" else nv.NVKV_KV_BF16
     shards = [nv.KVCache(wl.B, wl.H, wl.grid_h, wl.grid_w, wl.C, wl.S, wl.W, dtype,
                          shard_rank=r, shard_count=count) for r in range(count)]
     ts = wl.T // count
-    assert all(c.rows == (wl.S + wl.W) * ts for c in shards)
+    tr = ts + (ts & 1)                    # rows per slot: one padding row if ts is odd
+    assert all(c.rows == (wl.S + wl.W) * tr for c in shards)
     ora = OracleStream(wl, seed=2, keep_inputs=(kv == "bf16"))
     quantized = kv == "nvfp4"
     for step in range(1, steps + 1):
@@ -50,8 +61,9 @@ def test_shards_bit_exact_and_merge_to_whole_attention(name, count, kv, steps):
             lses.append(lse)
         merged_lse = torch.empty(wl.B, wl.H, wl.Lq, dtype=torch.float32, device="cuda")
         merged = nv.lse_merge(outs, lses, lse_out=merged_lse)
-        # rank 1's query slice alone: the same rows as the full merge, bit for bit
-        q0, q1 = wl.Lq // count, 2 * wl.Lq // count
+        # rank 1's query slice alone (the last rows for one shard): the same
+        # rows as the full merge, bit for bit
+        q0, q1 = (wl.Lq // count, 2 * wl.Lq // count) if count > 1 else (wl.Lq // 2, wl.Lq)
         part = nv.lse_merge(outs, lses, q0, q1)
         torch.cuda.synchronize()
         assert all(c.device_status() == 0 for c in shards)
@@ -64,7 +76,7 @@ def test_shards_bit_exact_and_merge_to_whole_attention(name, count, kv, steps):
                 for fid in new[b]:
                     p = _slot_of(c, b, fid)
                     e = ora.frame(b, fid)
-                    rows = slice(p * ts, (p + 1) * ts)
+                    rows = slice(p * tr, p * tr + ts)
                     if quantized:
                         for w in ("k", "v"):
                             assert np.array_equal(c.codes(w)[b, :, rows].cpu().numpy(),
@@ -177,3 +189,78 @@ def test_sequence_parallel_class_on_one_rank():
         del sp
     finally:
         dist.destroy_process_group()
+
+
+def _merge_inputs(n, B=1, Lq=200, H=3, seed=0):
+    gen = torch.Generator().manual_seed(seed)
+    o = [torch.randn(B, Lq, H, 128, generator=gen).to(torch.bfloat16).cuda() for _ in range(n)]
+    lse = [(torch.randn(B, H, Lq, generator=gen) * 3).cuda() for _ in range(n)]
+    return o, lse
+
+
+def test_synced_merge_after_peer_signal():
+    """Rank 0 of 2, with rank 1's signal for epoch 1 already in rank 0's flag
+    array (stored by the host, standing in for rank 1's kernel): the synced
+    merge signals rank 1, passes the barrier and returns what the plain merge
+    returns, bit for bit; the status stays 0."""
+    import nvfp4_kv_cache_append_b200 as nv
+    from nvfp4_kv_cache_append_b200 import _lib as L
+    o, lse = _merge_inputs(2)
+    B, Lq, H = 1, 200, 3
+    flags = [torch.zeros(16, dtype=torch.int32, device="cuda") for _ in range(2)]
+    flags[0][1] = 1
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.empty(B, 100, H, 128, dtype=torch.bfloat16, device="cuda")
+    L.nvkv_lse_merge_synced([t.data_ptr() for t in o], [t.data_ptr() for t in lse],
+                            [f.data_ptr() for f in flags], 0, 1, 2_000_000, status.data_ptr(),
+                            B, H, Lq, 0, 100, out.data_ptr())
+    want = nv.lse_merge(o, lse, 0, 100)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.equal(out, want)
+    assert flags[1][0].item() == 1 and flags[0][0].item() == 1     # rank 0 signalled both
+
+
+def test_synced_merge_times_out_without_signal():
+    """No rank 1 signal ever arrives: the wait runs out after 0.3 s, the kernel
+    writes NVKV_ERR_TIMEOUT to the status word and returns; the context stays
+    usable (a plain merge afterwards gives the right answer)."""
+    import nvfp4_kv_cache_append_b200 as nv
+    from nvfp4_kv_cache_append_b200 import _lib as L
+    o, lse = _merge_inputs(2, seed=1)
+    B, Lq, H = 1, 200, 3
+    flags = [torch.zeros(16, dtype=torch.int32, device="cuda") for _ in range(2)]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.empty(B, Lq, H, 128, dtype=torch.bfloat16, device="cuda")
+    L.nvkv_lse_merge_synced([t.data_ptr() for t in o], [t.data_ptr() for t in lse],
+                            [f.data_ptr() for f in flags], 0, 1, 300_000, status.data_ptr(),
+                            B, H, Lq, 0, Lq, out.data_ptr())
+    torch.cuda.synchronize()
+    assert int(status.item()) == L.STATUS_CODE["NVKV_ERR_TIMEOUT"]
+    assert flags[1][0].item() == 1                                 # the signal went out first
+    again = nv.lse_merge(o, lse)
+    ref_o, _ = oracle_lse_merge([t.float().cpu().numpy() for t in o],
+                                [t.cpu().permute(0, 2, 1).double().numpy() for t in lse])
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(again.float().cpu().numpy(), ref_o, rtol=1e-2, atol=1e-2)
+
+
+def test_synced_merge_rejects_bad_arguments():
+    from nvfp4_kv_cache_append_b200 import _lib as L
+    o, lse = _merge_inputs(2)
+    flags = [torch.zeros(16, dtype=torch.int32, device="cuda") for _ in range(2)]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.empty(1, 200, 3, 128, dtype=torch.bfloat16, device="cuda")
+    op, lp, fp = [t.data_ptr() for t in o], [t.data_ptr() for t in lse], [f.data_ptr() for f in flags]
+    for rank, epoch, timeout, fl, st in [(2, 1, 1000, fp, status.data_ptr()),
+                                         (0, 0, 1000, fp, status.data_ptr()),
+                                         (0, 1, 0, fp, status.data_ptr()),
+                                         (0, 1, 1000, [fp[0], 0], status.data_ptr()),
+                                         (0, 1, 1000, fp, 0)]:
+        with pytest.raises(L.NvkvError):
+            L.nvkv_lse_merge_synced(op, lp, fl, rank, epoch, timeout, st, 1, 3, 200, 0, 200,
+                                    out.data_ptr())
+    with pytest.raises(L.NvkvError):
+        L.nvkv_lse_merge_synced(op, lp, [fp[0] + 2, fp[1]], 0, 1, 1000, status.data_ptr(), 1, 3,
+                                200, 0, 200, out.data_ptr())
+    assert int(status.item()) == 0

@@ -62,7 +62,7 @@ def _worker(rank, world, port, errq):
         raise
 
 
-@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("world", [2, 4, 8])
 def test_sp_plans_and_merge_over_gloo(world):
     port = _free_port()
     ctx = mp.get_context("spawn")
