@@ -75,6 +75,27 @@ def lib():
             L.oracle_attention_rows.argtypes = [f32p, f64p, f64p, ctypes.c_int64, i32p, i32p, i32p,
                                                 i32p, i64p, ctypes.c_int64, ctypes.c_int, i32p,
                                                 ctypes.c_double, f64p, f64p]
+            fp = ctypes.POINTER(ctypes.c_float)
+            L.oracle_rope_cs_f32.restype = None
+            L.oracle_rope_cs_f32.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_double, fp, fp]
+            L.oracle_rope3d_f32.restype = None
+            L.oracle_rope3d_f32.argtypes = [f32p, i32p, i32p, ctypes.c_double]
+            L.oracle_k_spatial_rope_f32.restype = None
+            L.oracle_k_spatial_rope_f32.argtypes = [f32p, ctypes.c_int64, i32p, ctypes.c_int, i32p,
+                                                    ctypes.c_double]
+            L.oracle_q_row_global_scale.restype = ctypes.c_float
+            L.oracle_q_row_global_scale.argtypes = [f32p]
+            L.oracle_q_for_frame.restype = None
+            L.oracle_q_for_frame.argtypes = [f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, i32p,
+                                             ctypes.c_double, ctypes.c_float, u8p, u8p]
+            L.oracle_fp4_dot.restype = ctypes.c_double
+            L.oracle_fp4_dot.argtypes = [u8p, u8p, ctypes.c_float, u8p, u8p, ctypes.c_float]
+            L.oracle_attention_rows_fp4qk.restype = None
+            L.oracle_attention_rows_fp4qk.argtypes = [f32p, f64p, f64p, ctypes.c_int64, i32p,
+                                                      i32p, i32p, i64p, ctypes.c_int64,
+                                                      ctypes.c_int, i32p, ctypes.c_double,
+                                                      ctypes.c_int, f64p, f64p]
             L.oracle_block_scale_code.restype = ctypes.c_uint8
             L.oracle_block_scale_code.argtypes = [ctypes.c_float]
             L.oracle_e2m1_encode_array.restype = None
@@ -204,4 +225,77 @@ def attention_rows(q, k: np.ndarray, v: np.ndarray, k_frame_pos, k_tok, q_frame_
                                 np.ascontiguousarray(q_frame_pos, np.int32),
                                 np.ascontiguousarray(q_tok, np.int32), rows, rows.size, int(grid_w),
                                 np.asarray(split, np.int32), float(base), out, lse)
+    return out, lse
+
+
+# ------------------------------------------ block-scaled FP4 Q K^T (a reading)
+# The steps and their precision are stated in nvfp4_oracle.c, section
+# "block-scaled FP4 Q K^T (a reading)".
+
+def rope_cs_f32(pos: int, i: int, d: int, base: float = ROPE_BASE):
+    """cos and sin of pair i of a width-d segment at position pos, each rounded to float."""
+    c, s = ctypes.c_float(), ctypes.c_float()
+    lib().oracle_rope_cs_f32(int(pos), int(i), int(d), float(base), ctypes.byref(c), ctypes.byref(s))
+    return np.float32(c.value), np.float32(s.value)
+
+
+def rope3d_f32(x, pos3, split=ROPE_SPLIT, base=ROPE_BASE) -> np.ndarray:
+    """One 128-vector rotated in float (the quantizer-feeding rotation)."""
+    v = _as_f32(x).reshape(128).copy()
+    lib().oracle_rope3d_f32(v, np.asarray(pos3, np.int32), np.asarray(split, np.int32), float(base))
+    return v
+
+
+def k_spatial_rope_f32(k, tok, grid_w: int, split=ROPE_SPLIT, base=ROPE_BASE) -> np.ndarray:
+    """K rows [n, 128] with their h and w segments rotated at each row's token."""
+    a = _as_f32(k).reshape(-1, 128).copy()
+    t = np.ascontiguousarray(tok, np.int32).reshape(-1)
+    assert t.size == a.shape[0]
+    if a.shape[0]:
+        lib().oracle_k_spatial_rope_f32(a, a.shape[0], t, int(grid_w), np.asarray(split, np.int32),
+                                        float(base))
+    return a
+
+
+def q_row_global_scale(q) -> float:
+    a = _as_f32(q).reshape(128)
+    return float(lib().oracle_q_row_global_scale(a))
+
+
+def q_for_frame(q, dpos: int, q_tok: int, grid_w: int, s_gq: float, split=ROPE_SPLIT,
+                base=ROPE_BASE):
+    """Q_fk of one row for relative frame index dpos: (codes [64], scales [8])."""
+    a = _as_f32(q).reshape(128)
+    codes = np.zeros(64, np.uint8)
+    scales = np.zeros(8, np.uint8)
+    lib().oracle_q_for_frame(a, int(dpos), int(q_tok), int(grid_w), np.asarray(split, np.int32),
+                             float(base), float(np.float32(s_gq)), codes, scales)
+    return codes, scales
+
+
+def fp4_dot(ca, sa, ga: float, cb, sb, gb: float) -> float:
+    """Block form of one FP4 x FP4 dot product (integer code sums x block scales)."""
+    f = lambda x: np.ascontiguousarray(x, np.uint8)
+    return float(lib().oracle_fp4_dot(f(ca), f(sa), float(np.float32(ga)), f(cb), f(sb),
+                                      float(np.float32(gb))))
+
+
+def attention_rows_fp4qk(q, k: np.ndarray, v: np.ndarray, k_frame_pos, q_frame_pos, q_tok, rows,
+                         grid_w: int, quantize_q: bool = True, split=ROPE_SPLIT, base=ROPE_BASE):
+    """Chunk attention of one (batch, head) with FP4 logits: q [Lq, 128]
+    pre-RoPE, k [Lk, 128] the cached K' rows dequantized (spatially rotated
+    keys, quantized), v [Lk, 128] fp64.  ``quantize_q=False`` keeps Q_fk in
+    float.  Returns (out [n, 128], lse [n])."""
+    qa = _as_f32(q).reshape(-1, 128)
+    ka = np.ascontiguousarray(k, np.float64).reshape(-1, 128)
+    va = np.ascontiguousarray(v, np.float64).reshape(-1, 128)
+    Lk = ka.shape[0]
+    rows = np.ascontiguousarray(rows, np.int64)
+    out = np.zeros((rows.size, 128), np.float64)
+    lse = np.zeros(rows.size, np.float64)
+    lib().oracle_attention_rows_fp4qk(qa, ka, va, Lk, np.ascontiguousarray(k_frame_pos, np.int32),
+                                      np.ascontiguousarray(q_frame_pos, np.int32),
+                                      np.ascontiguousarray(q_tok, np.int32), rows, rows.size,
+                                      int(grid_w), np.asarray(split, np.int32), float(base),
+                                      1 if quantize_q else 0, out, lse)
     return out, lse

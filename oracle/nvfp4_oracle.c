@@ -260,6 +260,199 @@ void oracle_attention_rows(const float *q, const double *k, const double *v, int
     free(kr);
 }
 
+/* ------------------------------------- block-scaled FP4 Q K^T (a reading) */
+
+/* A reading of "NVFP4 quantization end to end" (evermx.com, heading "NVFP4
+ * Quantization End-to-End": the KV cache is held in the same 4-bit format as
+ * the W4A4 generator) for the logits: Q K^T taken on FP4 operands, as a
+ * block-scaled tensor-core contraction would, instead of on dequantized K.
+ * The pages give no such kernel; the steps below are the plainest reading
+ * that keeps the relative 3D RoPE ("NVlabs LongLive", refft.com, Core
+ * Analysis block on KV-cache relative RoPE) exact:
+ *  1. At append, K's spatial pairs (h and w segments) are rotated at the
+ *     token's (h, w); its frame segment is stored unrotated.  The rotated row
+ *     is quantized with the cache's NVFP4 rules (s_g from the first chunk's
+ *     amax of the rotated rows).
+ *  2. A query row at frame index f_q and (h_q, w_q) meets the keys of a frame
+ *     at index f_k through Q_fk: its frame segment rotated by the relative
+ *     index f_q - f_k, its spatial segments at (h_q, w_q).  Then
+ *     Q_fk . K' = R(f_q, h_q, w_q) q . R(f_k, h_k, w_k) k exactly in real
+ *     arithmetic, since the frame rotations of q and k combine to their
+ *     difference and K' carries k's spatial rotation.
+ *  3. Q_fk is quantized with the NVFP4 rules, one global scale per query row
+ *     that holds for every rotation: s_gq = fl32(p / 2688) with p the row's
+ *     largest pair magnitude fl32(sqrt(fl32(fl32(x^2) + fl32(y^2)))) (a
+ *     rotation keeps each pair's magnitude, so no element of any Q_fk exceeds
+ *     it but by rounding, which the 448 and 6 clamps absorb).
+ *  4. The logit is the dot product of the dequantized Q_fk and K' rows, over
+ *     sqrt(128); the softmax and the weighted sum of V are unchanged.
+ * Precision: the rotations feed a quantizer whose codes are integers, so
+ * they are fixed in float: cos and sin of the fp64 angle pos * base^(-2i/d),
+ * each rounded once to float, and (fl32(fl32(x c) - fl32(y s)),
+ * fl32(fl32(x s) + fl32(y c))).  Everything after dequantization is fp64. */
+
+static float f32_add(float a, float b) { return (float)((double)a + (double)b); }
+static float f32_sub(float a, float b) { return (float)((double)a - (double)b); }
+
+/* cos and sin of pair i of a RoPE segment of width d at integer position pos,
+ * each rounded once to float. */
+void oracle_rope_cs_f32(int pos, int i, int d, double base, float *c, float *s)
+{
+    double a = (double)pos * pow(base, -2.0 * i / (double)d);
+    *c = (float)cos(a);
+    *s = (float)sin(a);
+}
+
+/* One pair (x, y) rotated in float with the rounded cos c and sin s. */
+static void rot_pair_f32(float *x, float *y, float c, float s)
+{
+    float x0 = *x, y0 = *y;
+    *x = f32_sub(f32_mul(x0, c), f32_mul(y0, s));
+    *y = f32_add(f32_mul(x0, s), f32_mul(y0, c));
+}
+
+/* Rotate the channels of one 128-vector in float, segment by segment, at
+ * positions pos3 (frame, h, w); a position of 0 leaves its segment as is. */
+void oracle_rope3d_f32(float *x, const int *pos3, const int *split, double base)
+{
+    int off = 0;
+    for (int ax = 0; ax < 3; ++ax) {
+        int d = split[ax];
+        if (pos3[ax] != 0)
+            for (int i = 0; i < d / 2; ++i) {
+                float c, s;
+                oracle_rope_cs_f32(pos3[ax], i, d, base, &c, &s);
+                rot_pair_f32(&x[off + 2 * i], &x[off + 2 * i + 1], c, s);
+            }
+        off += d;
+    }
+}
+
+/* Step 1: K rows (bf16 values as float) with their spatial segments rotated
+ * at each row's token (h = tok / grid_w, w = tok % grid_w), in place. */
+void oracle_k_spatial_rope_f32(float *k, int64_t n, const int *tok, int grid_w, const int *split,
+                               double base)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n; ++r) {
+        int pos3[3] = {0, tok[r] / grid_w, tok[r] % grid_w};
+        oracle_rope3d_f32(k + r * 128, pos3, split, base);
+    }
+}
+
+/* Step 3: the per-row global scale of Q (1 if not a normal float). */
+float oracle_q_row_global_scale(const float *q)
+{
+    float p = 0.0f;
+    for (int i = 0; i < 64; ++i) {
+        float x = q[2 * i], y = q[2 * i + 1];
+        float m = (float)sqrt((double)f32_add(f32_mul(x, x), f32_mul(y, y)));
+        if (m > p) p = m;
+    }
+    float s = f32_div(p, 2688.0f);
+    if (!(s >= 1.17549435e-38f)) s = 1.0f;
+    return s;
+}
+
+/* Steps 2 and 3 for one query row and one relative frame index dpos:
+ * Q_fk quantized (codes [64], scales [8]) with the row's global scale. */
+void oracle_q_for_frame(const float *q, int dpos, int q_tok, int grid_w, const int *split,
+                        double base, float s_gq, uint8_t *codes, uint8_t *scales)
+{
+    float x[128];
+    memcpy(x, q, sizeof(x));
+    int pos3[3] = {dpos, q_tok / grid_w, q_tok % grid_w};
+    oracle_rope3d_f32(x, pos3, split, base);
+    oracle_quantize_rows(x, 1, s_gq, codes, scales);
+}
+
+/* The block form of one FP4 logit as a block-scaled contraction forms it:
+ * per 16-element block the integer sum of code products (E2M1 values are
+ * multiples of 1/2, so 4 times each product is an integer), times the two
+ * block scales; then the global scales.  Equal to the dot product of the
+ * dequantized rows up to fp64 rounding. */
+double oracle_fp4_dot(const uint8_t *ca, const uint8_t *sa, float ga, const uint8_t *cb,
+                      const uint8_t *sb, float gb)
+{
+    double acc = 0.0;
+    for (int blk = 0; blk < 8; ++blk) {
+        long long isum = 0;
+        for (int i = blk * 16; i < blk * 16 + 16; ++i) {
+            uint8_t qa = (ca[i / 2] >> ((i & 1) * 4)) & 15, qb = (cb[i / 2] >> ((i & 1) * 4)) & 15;
+            isum += (long long)llround(4.0 * oracle_e2m1_decode(qa) * oracle_e2m1_decode(qb));
+        }
+        acc += (double)isum * 0.25 * oracle_e4m3_decode(sa[blk]) * oracle_e4m3_decode(sb[blk]);
+    }
+    return acc * (double)ga * (double)gb;
+}
+
+/* Step 4: chunk attention of one (batch, head) on the listed query rows with
+ * FP4 logits.  q [Lq][128] pre-RoPE query values; kd [Lk][128] the cached K'
+ * rows dequantized (step 1; exact in fp64); v [Lk][128] dequantized values;
+ * positions as in oracle_attention_rows.  Q_fk is formed once per distinct
+ * key frame index; quantize_q = 0 keeps it in float (no step 3), which the
+ * tests use to check the RoPE split on its own.  out [n_rows][128], lse
+ * [n_rows]. */
+void oracle_attention_rows_fp4qk(const float *q, const double *kd, const double *v, int64_t Lk,
+                                 const int *k_frame_pos, const int *q_frame_pos, const int *q_tok,
+                                 const int64_t *rows, int64_t n_rows, int grid_w, const int *split,
+                                 double base, int quantize_q, double *out, double *lse)
+{
+    int max_pos = 0;
+    for (int64_t j = 0; j < Lk; ++j)
+        if (k_frame_pos[j] > max_pos) max_pos = k_frame_pos[j];
+    const double scale = 1.0 / sqrt(128.0);
+    #pragma omp parallel
+    {
+        double *logit = (double *)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+        double *qd = (double *)malloc(sizeof(double) * (size_t)(max_pos + 1) * 128);
+        char *have = (char *)malloc((size_t)max_pos + 1);
+        #pragma omp for schedule(dynamic, 1)
+        for (int64_t ri = 0; ri < n_rows; ++ri) {
+            int64_t r = rows[ri];
+            const float *qr = q + r * 128;
+            float s_gq = oracle_q_row_global_scale(qr);
+            memset(have, 0, (size_t)max_pos + 1);
+            double m = -INFINITY;
+            for (int64_t j = 0; j < Lk; ++j) {
+                int fk = k_frame_pos[j];
+                if (!have[fk]) {
+                    if (quantize_q) {
+                        uint8_t c[64], sc[8];
+                        oracle_q_for_frame(qr, q_frame_pos[r] - fk, q_tok[r], grid_w, split,
+                                           base, s_gq, c, sc);
+                        oracle_dequant_rows(c, sc, 1, s_gq, qd + (size_t)fk * 128);
+                    } else {
+                        float x[128];
+                        memcpy(x, qr, sizeof(x));
+                        int pos3[3] = {q_frame_pos[r] - fk, q_tok[r] / grid_w, q_tok[r] % grid_w};
+                        oracle_rope3d_f32(x, pos3, split, base);
+                        for (int i = 0; i < 128; ++i) qd[(size_t)fk * 128 + i] = (double)x[i];
+                    }
+                    have[fk] = 1;
+                }
+                double s = 0.0;
+                for (int i = 0; i < 128; ++i) s += qd[(size_t)fk * 128 + i] * kd[j * 128 + i];
+                logit[j] = s * scale;
+                if (logit[j] > m) m = logit[j];
+            }
+            double acc[128];
+            for (int i = 0; i < 128; ++i) acc[i] = 0.0;
+            double l = 0.0;
+            for (int64_t j = 0; j < Lk; ++j) {
+                double p = exp(logit[j] - m);
+                l += p;
+                for (int i = 0; i < 128; ++i) acc[i] += p * v[j * 128 + i];
+            }
+            for (int i = 0; i < 128; ++i) out[ri * 128 + i] = (Lk > 0) ? acc[i] / l : 0.0;
+            if (lse) lse[ri] = (Lk > 0) ? m + log(l) : -INFINITY;
+        }
+        free(have);
+        free(qd);
+        free(logit);
+    }
+}
+
 /* ------------------------------------------------------ array entry points */
 
 /* Block-scale code for a scale ratio t (the clamp at 448 included). */

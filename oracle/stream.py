@@ -7,6 +7,11 @@ their own frames included).  Keys are cached before RoPE and rotated at read
 time, following "NVlabs LongLive" (refft.com), Core Analysis block "How do
 KV-cache relative RoPE and TriAttention work together".
 
+With ``fp4_qk=True`` the stream follows the block-scaled FP4 Q K^T reading
+(``nvfp4_oracle.c``, section "block-scaled FP4 Q K^T (a reading)"): K is
+cached with its spatial RoPE applied before quantization and the logits are
+taken between FP4 Q (rotated per key frame) and the cached FP4 K.
+
 Inputs come from ``kvsynth`` only; no value comes from the CUDA path.
 """
 from __future__ import annotations
@@ -16,14 +21,17 @@ from typing import Dict, List, Optional, Tuple
 import numpy as np
 
 import kvsynth
-from . import amax as _amax, attention_rows, dequant_rows, global_scale, quantize_rows
+from . import (amax as _amax, attention_rows, attention_rows_fp4qk, dequant_rows, global_scale,
+               k_spatial_rope_f32, quantize_rows)
 from .ring import OracleRing
 
 
 class OracleStream:
     def __init__(self, wl: kvsynth.Workload, seed: int = 0,
-                 shot_sched: Optional[List[List[int]]] = None, keep_inputs: bool = True):
+                 shot_sched: Optional[List[List[int]]] = None, keep_inputs: bool = True,
+                 fp4_qk: bool = False):
         self.wl = wl
+        self.fp4_qk = fp4_qk
         self.seed = seed
         self.rings = [OracleRing(wl.S, wl.W, wl.C) for _ in range(wl.B)]
         self.sched = shot_sched if shot_sched is not None else kvsynth.shot_schedule(wl, seed)
@@ -35,14 +43,25 @@ class OracleStream:
 
     # ------------------------------------------------------------ append
 
+    def _k_rows(self, kf, b, h, sl=None):
+        """K rows [n, 128] of (b, h) over chunk rows ``sl`` as the cache
+        quantizes them: as given, or spatially rotated (``fp4_qk``)."""
+        wl = self.wl
+        sl = slice(0, wl.Lq) if sl is None else sl
+        rows = np.ascontiguousarray(kf[b, sl, h, :])
+        if not self.fp4_qk:
+            return rows
+        tok = (np.arange(wl.Lq, dtype=np.int32) % wl.T)[sl]
+        return k_spatial_rope_f32(rows, tok, wl.grid_w)
+
     def _scales_from(self, k, v) -> np.ndarray:
         wl = self.wl
         s = np.zeros((2, wl.B, wl.H), np.float32)
-        for t, x in enumerate((k, v)):
-            xf = x.float().numpy()
-            for b in range(wl.B):
-                for h in range(wl.H):
-                    s[t, b, h] = global_scale(_amax(np.ascontiguousarray(xf[b, :, h, :])))
+        kf, vf = k.float().numpy(), v.float().numpy()
+        for b in range(wl.B):
+            for h in range(wl.H):
+                s[0, b, h] = global_scale(_amax(self._k_rows(kf, b, h)))
+                s[1, b, h] = global_scale(_amax(np.ascontiguousarray(vf[b, :, h, :])))
         return s
 
     def step(self, k=None, v=None, q=None):
@@ -104,7 +123,8 @@ class OracleStream:
                 codes = np.zeros((wl.H, wl.T, 64), np.uint8)
                 scales = np.zeros((wl.H, wl.T, 8), np.uint8)
                 for h in range(wl.H):
-                    codes[h], scales[h] = quantize_rows(rows[h], self.s_g[t, b, h])
+                    src = self._k_rows(kf, b, h, sl) if name == "k" else rows[h]
+                    codes[h], scales[h] = quantize_rows(src, self.s_g[t, b, h])
                 ent[name + "_codes"] = codes
                 ent[name + "_scales"] = scales
                 if self.keep_inputs:
@@ -151,7 +171,10 @@ class OracleStream:
     def attention(self, b: int, h: int, rows, quantized: bool = True, tokens=None):
         """Oracle outputs (fp64) for query rows ``rows`` of (b, h) at the current
         step: (out [n, 128], lse [n]); ``tokens`` as in ``visible_kv``."""
-        k, v, fpos, tok = self.visible_kv(b, h, quantized, tokens)
         qpos, qtok = self.query_positions(b)
         q = self.q[b, :, h, :]
+        if self.fp4_qk and quantized:
+            k, v, fpos, _ = self.visible_kv(b, h, True, tokens)     # K' dequantized
+            return attention_rows_fp4qk(q, k, v, fpos, qpos, qtok, rows, self.wl.grid_w)
+        k, v, fpos, tok = self.visible_kv(b, h, quantized, tokens)
         return attention_rows(q, k, v, fpos, tok, qpos, qtok, rows, self.wl.grid_w)
