@@ -461,6 +461,9 @@ def run_ours(args):
             "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": gbs / peaks["hbm_gbs"], "kernel": "k_nvfp4_append" if fp4 else "k_bf16_append",
             "us_per_launch": us,
+            "traffic": _ncu_traffic("k_nvfp4_append", wl.name) if fp4 else None,
+            "traffic_note": "ncu DRAM bytes of one cold launch; the codes and scales it writes "
+                            "stay in L2, so only the bf16 reads show",
             "timing": "isolated, cold L2: 40 x (256 MB flush + append) minus 40 x flush, median of 5"}
     if ws == 1 and not args.no_extra:
         clocks2 = ClockSampler(local)
@@ -785,7 +788,10 @@ def cpu_baseline(wl, seconds=20.0):
     import oracle
     oracle.build()
     sample = OracleSample(wl)
-    n_rows = max(8, int(seconds * 6))
+    # a pilot of 8 rows sizes the sample to about `seconds` of oracle work
+    _, t_app, t_att = sample.run(wl.Lq, 8)
+    per_row = max(t_att / 8, 1e-6)
+    n_rows = int(max(8, min(wl.Lq, (seconds - t_app) / per_row)))
     value, t_app, t_att = sample.run(wl.Lq, n_rows)
     return {"value": value, "unit": "query tok/s", "cores": _oracle_cores(), "kind": "oracle",
             "sample": f"one {wl.name} step: full-chunk quantize ({wl.Lq} tokens x {wl.H} heads, "
