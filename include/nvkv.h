@@ -309,7 +309,10 @@ NVKV_API size_t nvkv_attention_workspace_bytes(const nvkv_desc *desc);
  * workspace: device memory of nvkv_attention_workspace_bytes() bytes (else
  * NVKV_ERR_CAPACITY).  NVKV_ERR_STATE if nothing was appended yet;
  * NVKV_ERR_UNSUPPORTED for a RoPE
- * split other than 44/42/42 or grid_h or grid_w above 256. */
+ * split other than 44/42/42, grid_h or grid_w above 256, or RoPE tables too
+ * large for one CTA's shared memory: 176 (frames resident) + 168 (grid_h +
+ * grid_w) bytes above about 104 KB (only near the largest grids with many
+ * frames). */
 NVKV_API nvkv_status chunk_attention_nvfp4kv(const nvkv_desc *desc, const nvkv_cache *cache,
                                     const nvkv_ring *ring, const void *q, void *out, float *lse,
                                     void *workspace, size_t workspace_bytes, nvkv_stream stream);

@@ -278,6 +278,7 @@ nvkv_status attention_common(const nvkv_desc *desc, const nvkv_cache *cache,
         a.q_pos0[b] = s.n_resident - desc->C;
         if (s.n_resident > a.n_fpos) a.n_fpos = s.n_resident;
     }
+    if (!nvkv::attention_fits(a)) return NVKV_ERR_UNSUPPORTED;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return NVKV_ERR_CUDA;
     const int dev_slots = nvkv::attention_slots(dev);

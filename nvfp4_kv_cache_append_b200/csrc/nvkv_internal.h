@@ -86,6 +86,8 @@ size_t attention_workspace_bytes(int n_slots);
 int attention_slots(int device);     // CTA pairs that can be resident at once
 
 cudaError_t launch_chunk_attention(const AttnLaunch &a, cudaStream_t s);
+// whether the kernel's shared memory (with the launch's RoPE tables) fits a CTA
+bool attention_fits(const AttnLaunch &a);
 
 // K/V projection of one chunk (x [M][hidden] times W^T, W [H*128][hidden],
 // bf16 in, f32 accumulate), its epilogue writing bf16 K/V (mode 0) or the

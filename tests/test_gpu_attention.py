@@ -167,3 +167,15 @@ def test_q_small(kv_dtype):
 def test_q_large_bf16kv():
     """The twin with Q times 2^12 and K times 2^-12 (K stays inside f16)."""
     _scaled_run(kvsynth.WORKLOADS["tiny"], 1, 2.0 ** 12, 2.0 ** -12)
+
+
+@pytest.mark.parametrize("kv_dtype", [0, 1], ids=["nvfp4", "bf16"])
+def test_round_robin_schedule_with_split_tail(kv_dtype):
+    """192 work items (2 streams x 32 heads x 3 query-tile pairs) of 14 key
+    tiles on 74 CTA pairs: one round of whole items round-robin, then the
+    other 118 items' tiles cut end to end, so that most of them are split
+    between two pairs and merged through partial records.  Every row of
+    sampled heads against the oracle."""
+    wl = kvsynth.Workload("rr", B=2, H=32, D=128, grid_h=16, grid_w=16, C=3, S=1, W=6, steps=3)
+    _run(wl, kv_dtype, {1, wl.steps}, lambda wl, s, b, h: np.arange(wl.Lq),
+         lambda wl, s, b: range(b, wl.H, 5))
