@@ -788,9 +788,11 @@ def cpu_baseline(wl, seconds=20.0):
     import oracle
     oracle.build()
     sample = OracleSample(wl)
-    # a pilot of 8 rows sizes the sample to about `seconds` of oracle work
-    _, t_app, t_att = sample.run(wl.Lq, 8)
-    per_row = max(t_att / 8, 1e-6)
+    # a pilot of 32 rows (after 8 that warm the thread pool) sizes the
+    # sample to about `seconds` of oracle work
+    sample.run(64, 8)
+    _, t_app, t_att = sample.run(wl.Lq, 32)
+    per_row = max(t_att / 32, 1e-6)
     n_rows = int(max(8, min(wl.Lq, (seconds - t_app) / per_row)))
     value, t_app, t_att = sample.run(wl.Lq, n_rows)
     return {"value": value, "unit": "query tok/s", "cores": _oracle_cores(), "kind": "oracle",
