@@ -579,7 +579,7 @@ def run_sp(args):
 
 def run_sp_emulate(args):
     """--sp-emulate: the per-rank kernel times of the sequence-parallel split
-    for N = 1, 2, 3, 4, 6 shards, all run on this one GPU: one shard's
+    for N = 1, 2, 3, 4, 6, 8 shards (those that divide T), all run on this one GPU: one shard's
     attention over its 1/N of every frame's tokens, and the merge of one
     rank's query slice from the N shards' partial results (local here; over
     NVLink on N GPUs).  L2 is flushed (256 MB written) before every timed
@@ -609,8 +609,8 @@ def run_sp_emulate(args):
         return statistics.median(ms)
 
     rows = []
-    for n in (1, 2, 3, 4, 6):
-        if wl.T % n or (wl.T // n) % 2:
+    for n in (1, 2, 3, 4, 6, 8):
+        if wl.T % n:
             continue
         shards = [nv.KVCache(wl.B, wl.H, wl.grid_h, wl.grid_w, wl.C, wl.S, wl.W, nv.NVKV_KV_NVFP4,
                              shard_rank=r, shard_count=n) for r in range(n)]
