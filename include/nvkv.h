@@ -262,6 +262,24 @@ NVKV_API nvkv_status nvfp4_kv_append_noalloc(const nvkv_desc *desc, const nvkv_c
                                              nvkv_ring *ring, const void *k, const void *v,
                                              nvkv_stream stream);
 
+/* Quantize-append for the block-scaled FP4 Q K^T reading (the KV cache "in
+ * the same format" as the W4A4 generator: evermx.com, heading "NVFP4
+ * Quantization End-to-End"; relative RoPE: "NVlabs LongLive", refft.com, Core
+ * Analysis block on KV-cache relative RoPE).  As nvfp4_kv_append, but each K
+ * row first has its spatial RoPE pairs (the 42-channel h and w segments)
+ * rotated at its token's (h, w), in float: cos and sin of the fp64 angle
+ * pos * rope_base^(-2i/42), each rounded once to float, and (fl(fl(x c) -
+ * fl(y s)), fl(fl(x s) + fl(y c))); the frame segment stays unrotated and V
+ * is appended as usual.  The first chunk's K amax is taken over the rotated
+ * rows.  The cache this fills holds keys for a contraction that applies only
+ * the frame rotation at read time; chunk_attention_nvfp4kv, which rotates
+ * the cached keys in all three segments, does not read it.
+ * NVKV_ERR_UNSUPPORTED unless the RoPE split is 44/42/42 and grid_h, grid_w
+ * <= 90; otherwise as nvfp4_kv_append. */
+NVKV_API nvkv_status nvfp4_kv_append_spatial_rope(const nvkv_desc *desc, const nvkv_cache *cache,
+                                                  nvkv_ring *ring, const void *k, const void *v,
+                                                  nvkv_stream stream);
+
 /* The bf16-KV twin: same slot logic, the chunk's bf16 K/V copied as is. */
 NVKV_API nvkv_status bf16_kv_append(const nvkv_desc *desc, const nvkv_cache *cache, nvkv_ring *ring,
                            const void *k, const void *v, nvkv_stream stream);

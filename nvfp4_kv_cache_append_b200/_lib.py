@@ -101,6 +101,7 @@ def _load():
         "nvfp4_kv_append": (i32, [D, C, R, vp, vp, vp]),
         "bf16_kv_append": (i32, [D, C, R, vp, vp, vp]),
         "nvfp4_kv_append_noalloc": (i32, [D, C, R, vp, vp, vp]),
+        "nvfp4_kv_append_spatial_rope": (i32, [D, C, R, vp, vp, vp]),
         "nvfp4_kv_overwrite": (i32, [D, C, R, vp, vp, vp]),
         "bf16_kv_overwrite": (i32, [D, C, R, vp, vp, vp]),
         "nvkv_attention_workspace_bytes": (sz, [D]),
@@ -250,6 +251,12 @@ def nvfp4_kv_append_noalloc(desc, cache, ring, k_ptr, v_ptr, stream=0) -> None:
     _check(lib.nvfp4_kv_append_noalloc(ctypes.byref(desc), ctypes.byref(cache),
                                        ctypes.byref(ring), k_ptr, v_ptr, stream),
            "nvfp4_kv_append_noalloc")
+
+
+def nvfp4_kv_append_spatial_rope(desc, cache, ring, k_ptr, v_ptr, stream=0) -> None:
+    _check(lib.nvfp4_kv_append_spatial_rope(ctypes.byref(desc), ctypes.byref(cache),
+                                            ctypes.byref(ring), k_ptr, v_ptr, stream),
+           "nvfp4_kv_append_spatial_rope")
 
 
 def bf16_kv_append(desc, cache, ring, k_ptr, v_ptr, stream=0) -> None:

@@ -135,6 +135,16 @@ class KVCache:
         fn = L.nvfp4_kv_append if self.fp4 else L.bf16_kv_append
         fn(self.desc, self.cache, self.ring, _ptr(k), _ptr(v), _stream(stream))
 
+    def append_spatial_rope(self, k: torch.Tensor, v: torch.Tensor, stream=None) -> None:
+        """Quantize-append with K's spatial RoPE applied first (the cache layout
+        of the block-scaled FP4 Q K^T reading; see nvfp4_kv_append_spatial_rope)."""
+        if not self.fp4:
+            raise ValueError("the spatial-RoPE append fills an NVFP4 cache")
+        self._check_io(k)
+        self._check_io(v)
+        L.nvfp4_kv_append_spatial_rope(self.desc, self.cache, self.ring, _ptr(k), _ptr(v),
+                                       _stream(stream))
+
     def overwrite(self, k: torch.Tensor, v: torch.Tensor, stream=None) -> None:
         """Denoising step: the newest chunk's K/V replaced in place (same slots)."""
         self._check_io(k)

@@ -152,6 +152,101 @@ __global__ void __launch_bounds__(1024) k_bf16_append(const __grid_constant__ Ap
     reinterpret_cast<uint4 *>(t ? a.v_data : a.k_data)[row * 16 + c] = ld_stream(src);
 }
 
+// ------------------------------------------- K with its spatial RoPE applied
+
+// Rotate the pairs of n consecutive channels starting at channel ch0 (even)
+// that lie in the h segment [44, 86) or the w segment [86, 128), in float:
+// (fl(fl(x c) - fl(y s)), fl(fl(x s) + fl(y c))), no contraction; the frame
+// segment [0, 44) is left as is.
+__device__ __forceinline__ void rotate_spatial(float *x, int n, int ch0, int hp, int wp,
+                                               const SpatialRope &R)
+{
+    for (int j = 0; j < n; j += 2) {
+        const int ch = ch0 + j;
+        if (ch < 44) continue;
+        const float2 cs = ch < 86 ? R.h[hp * 21 + ((ch - 44) >> 1)] : R.w[wp * 21 + ((ch - 86) >> 1)];
+        const float x0 = x[j], y0 = x[j + 1];
+        x[j] = __fsub_rn(__fmul_rn(x0, cs.x), __fmul_rn(y0, cs.y));
+        x[j + 1] = __fadd_rn(__fmul_rn(x0, cs.y), __fmul_rn(y0, cs.x));
+    }
+}
+
+// k_first_chunk_amax with K's spatial pairs rotated first (row l of the chunk
+// is token l % T of its frame, at (h, w) = divmod(l % T, grid_w))
+__global__ void k_first_chunk_amax_rope(const uint4 *__restrict__ k, const uint4 *__restrict__ v,
+                                        uint32_t *__restrict__ amax, int B, int H, int Lq, int T,
+                                        int grid_w, const __grid_constant__ SpatialRope R)
+{
+    __shared__ uint32_t s_max[64];
+    const int tid = threadIdx.y * blockDim.x + threadIdx.x;
+    if (tid < H) s_max[tid] = 0u;
+    __syncthreads();
+    const int t = blockIdx.y / B, b = blockIdx.y - t * B;
+    const uint4 *src = t ? v : k;
+    const int h = threadIdx.x >> 3, blk = threadIdx.x & 7;
+    float m = 0.0f;
+    for (int l = blockIdx.x * blockDim.y + threadIdx.y; l < Lq; l += gridDim.x * blockDim.y) {
+        const uint4 *p = src + (((size_t)b * Lq + l) * H + h) * 16 + blk * 2;
+        float x[16];
+        unpack_bf16x8(ld_stream(p), x);
+        unpack_bf16x8(ld_stream(p + 1), x + 8);
+        if (t == 0) {
+            const int tok = l % T;
+            rotate_spatial(x, 16, blk * 16, tok / grid_w, tok % grid_w, R);
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(x[i]));
+    }
+    uint32_t f = __float_as_uint(m);
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) {
+        const uint32_t g = __shfl_xor_sync(0xFFFFFFFFu, f, o);
+        f = g > f ? g : f;
+    }
+    if (blk == 0) atomicMax(&s_max[h], f);
+    __syncthreads();
+    if (tid < H && s_max[tid]) atomicMax(&amax[(t * B + b) * H + tid], s_max[tid]);
+}
+
+// k_nvfp4_append with K's spatial pairs rotated in float before quantizing
+// (the cache layout of the block-scaled FP4 Q K^T contraction); V as is.
+__global__ void __launch_bounds__(512) k_nvfp4_append_rope(const __grid_constant__ AppendLaunch a,
+                                                           const __grid_constant__ SpatialRope R)
+{
+    const int t = blockIdx.y / a.B, b = blockIdx.y - t * a.B;
+    const int l = blockIdx.x * blockDim.y + threadIdx.y;
+    if (l >= a.C * a.Ts) return;
+    const int h = threadIdx.x >> 2, pr = threadIdx.x & 3;
+    const int frame = frame_of(l, a), tok = l - frame * a.Ts;
+    const int src_l = frame * a.T + a.tok_off + tok;
+    const uint4 *src = reinterpret_cast<const uint4 *>(t ? a.v : a.k) +
+                       (((size_t)b * a.Lq + src_l) * a.H + h) * 16 + pr * 4;
+    const uint4 w0 = ld_stream(src), w1 = ld_stream(src + 1);
+    const uint4 w2 = ld_stream(src + 2), w3 = ld_stream(src + 3);
+    const int gi = (t * a.B + b) * a.H + h;
+    const float sg = head_scale(a, gi, l == 0 && pr == 0);
+    const int slot = a.slot[b * a.C + frame];
+    const size_t row = (size_t)(b * a.H + h) * a.R + (size_t)slot * a.Tr + tok;
+    if (t == 1) {
+        quantize_pair(a, t, h, pr, row, sg, w0, w1, w2, w3);
+        return;
+    }
+    float x[32];
+    unpack_bf16x8(w0, x);
+    unpack_bf16x8(w1, x + 8);
+    unpack_bf16x8(w2, x + 16);
+    unpack_bf16x8(w3, x + 24);
+    const int ft = a.tok_off + tok;
+    rotate_spatial(x, 32, pr * 32, ft / a.grid_w, ft % a.grid_w, R);
+    uint2 c0, c1;
+    const uint32_t s0 = quantize_block_f32(x, sg, c0);
+    const uint32_t s1 = quantize_block_f32(x + 16, sg, c1);
+    *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(a.k_data) + row * 64 + pr * 16) =
+        make_uint4(c0.x, c0.y, c1.x, c1.y);
+    *reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(a.k_scales) + row * 8 + pr * 2) =
+        (uint16_t)(s0 | (s1 << 8));
+}
+
 __global__ void k_encode_e2m1(const float *__restrict__ y, uint8_t *__restrict__ out, size_t n)
 {
     const size_t i0 = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
@@ -198,6 +293,26 @@ cudaError_t launch_nvfp4_append(const AppendLaunch &a_in, cudaStream_t s)
     }
     const dim3 grid((a.C * a.Ts + blk.y - 1) / blk.y, 2 * a.B);
     k_nvfp4_append<<<grid, blk, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_nvfp4_append_rope(const AppendLaunch &a_in, const SpatialRope &r, cudaStream_t s)
+{
+    AppendLaunch a = a_in;
+    a.inv_Ts = 1.0f / (float)a.Ts;
+    const dim3 blk = append_block(a.H, 4);
+    if (a.first) {
+        cudaError_t e = cudaMemsetAsync(a.amax, 0, sizeof(uint32_t) * 2 * a.B * a.H, s);
+        if (e != cudaSuccess) return e;
+        const dim3 blk8 = append_block(a.H, 8);
+        const unsigned gx = (a.Lq + blk8.y - 1) / blk8.y;
+        const dim3 g2(gx < 148 ? gx : 148, 2 * a.B);
+        k_first_chunk_amax_rope<<<g2, blk8, 0, s>>>(static_cast<const uint4 *>(a.k),
+                                                   static_cast<const uint4 *>(a.v), a.amax, a.B,
+                                                   a.H, a.Lq, a.T, a.grid_w, r);
+    }
+    const dim3 grid((a.C * a.Ts + blk.y - 1) / blk.y, 2 * a.B);
+    k_nvfp4_append_rope<<<grid, blk, 0, s>>>(a, r);
     return cudaGetLastError();
 }
 

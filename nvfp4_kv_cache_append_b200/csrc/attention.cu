@@ -677,7 +677,7 @@ __device__ void k_converter_role(Ctx &c)
 }
 
 // warps 8-11: this CTA's channel half of V for all 128 keys of each tile
-template <bool FP4, bool SHARD>
+template <bool FP4, bool SHARD, bool PAD>
 __device__ void v_converter_role(Ctx &c)
 {
     const AttnLaunch &a = *c.a;
@@ -694,7 +694,7 @@ __device__ void v_converter_role(Ctx &c)
             if (g >= 2 && !wait(c, B_VFREE + vb, ((g - 2) >> 1) & 1)) return;
             if (FP4) {
                 conv_v_fp4(stg, k, (int)c.rank,
-                           tile * BN + k < n_keys && (!SHARD || not_pad(a, tile * BN + k)), vdst);
+                           tile * BN + k < n_keys && (!PAD || not_pad(a, tile * BN + k)), vdst);
             } else {
                 const KeyPos kp = key_pos(c, sg.b, sg.h, n_keys, tile * BN + k, SHARD ? a.tok_off : 0);
                 conv_v_bf16(c, k, (int)c.rank, kp, vdst);
@@ -916,7 +916,7 @@ __device__ __forceinline__ void store_row_bf16(uint4 *dst, const float *acc, flo
     }
 }
 
-template <bool FP4, bool SHARD>
+template <bool FP4, bool PAD>
 __device__ void softmax_role(Ctx &c)
 {
     const AttnLaunch &a = *c.a;
@@ -967,7 +967,7 @@ __device__ void softmax_role(Ctx &c)
                     for (int i = 0; i < 32; ++i)
                         if (q * 32 + i >= nv) s[i] = -INFINITY;
                 }
-                if (SHARD && a.Tr != a.Tk) {
+                if (PAD) {
                     // padding keys (one per frame, key mod Tr == Tk) of this chunk
                     const int k0 = tile * BN + q * 32;
                     uint32_t pad = 0;
@@ -1122,8 +1122,9 @@ __device__ void softmax_role(Ctx &c)
 // ------------------------------------------------------------ kernel
 
 // VAR 0: a whole cache with an even number of tokens per frame; 1 (SHARD):
-// a shard whose first token is not token 0 of the frame, or whose slots hold
-// a padding row (odd token count); 2: the failure-path test.  Separate instantiations keep the
+// a shard whose first token is not token 0 of the frame; 3: a cache whose
+// slots hold a padding row (odd token count per frame), shard or not; 2: the
+// failure-path test.  Separate instantiations keep the
 // whole-cache kernel's code free of both.
 template <bool FP4, int VAR>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
@@ -1173,11 +1174,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     ptx::tc_fence_after();
 
     if (warp < 4) {
-        softmax_role<FP4, VAR == 1>(c);
+        softmax_role<FP4, VAR == 3>(c);
     } else if (warp < 8) {
-        k_converter_role<FP4, VAR == 1>(c);
+        k_converter_role<FP4, VAR == 1 || VAR == 3>(c);
     } else if (warp < 12) {
-        v_converter_role<FP4, VAR == 1>(c);
+        v_converter_role<FP4, VAR == 1 || VAR == 3, VAR == 3>(c);
     } else if (warp == 12) {
         if (FP4 && (threadIdx.x & 31) == 0) producer_role<VAR == 2>(c);
     } else if (warp == 13) {
@@ -1250,7 +1251,8 @@ cudaError_t launch_chunk_attention(const AttnLaunch &a, cudaStream_t s)
 {
     const bool fp4 = a.kv_dtype == NVKV_KV_NVFP4;
     if (fp4 && a.fault == NVKV_FAULT_SKIP_FIRST_STAGE && !a.tok_off) return launch<true, 2>(a, s);
-    if (a.tok_off || a.Tr != a.Tk) return fp4 ? launch<true, 1>(a, s) : launch<false, 1>(a, s);
+    if (a.Tr != a.Tk) return fp4 ? launch<true, 3>(a, s) : launch<false, 3>(a, s);
+    if (a.tok_off) return fp4 ? launch<true, 1>(a, s) : launch<false, 1>(a, s);
     return fp4 ? launch<true, 0>(a, s) : launch<false, 0>(a, s);
 }
 

@@ -85,6 +85,28 @@ __device__ __forceinline__ void unpack_bf16x8(uint4 a, float *x)
 // Codes of one 16-element block (bf16 in w0, w1) with global scale sg:
 // returns the E4M3 scale code, writes the 16 codes (element i in nibble i of
 // c.x | c.y << 32).
+// The same block rule for 16 float inputs (rotated keys), with IEEE division
+// for every quotient (the shared-divisor shortcut is only verified on bf16
+// inputs).
+__device__ __forceinline__ uint32_t quantize_block_f32(const float *x, float sg, uint2 &c)
+{
+    float amax16 = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax16 = fmaxf(amax16, fabsf(x[i]));
+    const float ratio = __fdiv_rn(amax16, __fmul_rn(6.0f, sg));
+    const uint32_t sb_code = e4m3_code(ratio);
+    const float sb = e4m3_value(sb_code);
+    c = make_uint2(0u, 0u);
+    if (sb == 0.0f) return sb_code;
+    const float d = __fmul_rn(sb, sg);
+    float y[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) y[i] = __fdiv_rn(x[i], d);
+    c.x = drop_negative_zero(e2m1x8(y));
+    c.y = drop_negative_zero(e2m1x8(y + 8));
+    return sb_code;
+}
+
 __device__ __forceinline__ uint32_t quantize_block(uint4 w0, uint4 w1, float sg, uint2 &c)
 {
     const float amax16 = halves_max(__vmaxu2(absmax_bits(w0), absmax_bits(w1)));

@@ -142,7 +142,7 @@ bool newest_chunk_slots(const nvkv_desc *d, const nvkv_ring *r, int32_t *slot_ou
 // cache->amax (which may then be null).
 nvkv_status append_common(const nvkv_desc *desc, const nvkv_cache *cache, const nvkv_ring *ring,
                           nvkv_ring *advance, const void *k, const void *v, cudaStream_t stream,
-                          int dtype, uint32_t *amax_scratch = nullptr)
+                          int dtype, uint32_t *amax_scratch = nullptr, bool spatial_rope = false)
 {
     const bool overwrite = advance == nullptr;
     nvkv_status st = check_desc(desc);
@@ -181,8 +181,26 @@ nvkv_status append_common(const nvkv_desc *desc, const nvkv_cache *cache, const 
     a.R = (int)rows_per_head(desc);
     a.C = desc->C;
     a.first = overwrite ? (ring->steps == 1 ? 1 : 0) : (ring->scales_fixed ? 0 : 1);
-    cudaError_t e = (dtype == NVKV_KV_NVFP4) ? nvkv::launch_nvfp4_append(a, stream)
-                                             : nvkv::launch_bf16_append(a, stream);
+    a.grid_w = desc->grid_w;
+    cudaError_t e;
+    if (spatial_rope) {
+        // cos and sin of each spatial pair: the fp64 angle pos * base^(-2i/42),
+        // cos and sin in fp64, each rounded once to float
+        static thread_local nvkv::SpatialRope r;
+        for (int ax = 0; ax < 2; ++ax) {
+            const int d = desc->rope_split[1 + ax], n = ax ? desc->grid_w : desc->grid_h;
+            float2 *tab = ax ? r.w : r.h;
+            for (int pos = 0; pos < n; ++pos)
+                for (int i = 0; i < d / 2; ++i) {
+                    const double ang = (double)pos * std::pow((double)desc->rope_base, -2.0 * i / (double)d);
+                    tab[pos * 21 + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+                }
+        }
+        e = nvkv::launch_nvfp4_append_rope(a, r, stream);
+    } else {
+        e = (dtype == NVKV_KV_NVFP4) ? nvkv::launch_nvfp4_append(a, stream)
+                                     : nvkv::launch_bf16_append(a, stream);
+    }
     if (e != cudaSuccess) return NVKV_ERR_CUDA;
     if (!overwrite) commit_append(desc, advance, a.slot);
     return NVKV_OK;
@@ -471,6 +489,19 @@ nvkv_status bf16_kv_append(const nvkv_desc *desc, const nvkv_cache *cache, nvkv_
                            const void *k, const void *v, nvkv_stream stream)
 {
     return append_common(desc, cache, ring, ring, k, v, (cudaStream_t)stream, NVKV_KV_BF16);
+}
+
+nvkv_status nvfp4_kv_append_spatial_rope(const nvkv_desc *desc, const nvkv_cache *cache,
+                                         nvkv_ring *ring, const void *k, const void *v,
+                                         nvkv_stream stream)
+{
+    nvkv_status st = check_desc(desc);
+    if (st != NVKV_OK) return st;
+    if (desc->rope_split[0] != 44 || desc->rope_split[1] != 42 || desc->rope_split[2] != 42 ||
+        desc->grid_h > nvkv::kRopeAppendMaxGrid || desc->grid_w > nvkv::kRopeAppendMaxGrid)
+        return NVKV_ERR_UNSUPPORTED;
+    return append_common(desc, cache, ring, ring, k, v, (cudaStream_t)stream, NVKV_KV_NVFP4,
+                         nullptr, true);
 }
 
 nvkv_status nvfp4_kv_overwrite(const nvkv_desc *desc, const nvkv_cache *cache,

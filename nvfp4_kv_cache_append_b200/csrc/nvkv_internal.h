@@ -21,8 +21,20 @@ struct AppendLaunch {
     int Tr;                          // rows per frame slot (Ts rounded up to even)
     float inv_Ts;                    // 1/Ts, set by the launchers (frame index by reciprocal)
     int first;                       // 1: measure amax and fix s_g
+    int grid_w;                      // tokens per latent row (spatial RoPE variant)
     int32_t slot[NVKV_MAX_BATCH * NVKV_MAX_CHUNK];  // [b * C + c] -> physical slot
 };
+
+// cos and sin (float) of the spatial RoPE pairs, for the append that rotates
+// K before quantizing it: h[pos * 21 + i] for pair i of the 42-channel h
+// segment at row pos, w[pos * 21 + i] likewise for the w segment.  Passed as
+// a kernel parameter (30 KB), which bounds the grid.
+constexpr int kRopeAppendMaxGrid = 90;
+struct SpatialRope {
+    float2 h[kRopeAppendMaxGrid * 21];
+    float2 w[kRopeAppendMaxGrid * 21];
+};
+cudaError_t launch_nvfp4_append_rope(const AppendLaunch &a, const SpatialRope &r, cudaStream_t s);
 
 // Tokens per frame of the cache a desc describes (the shard's share of each
 // frame) and the index of its first token within the frame.

@@ -227,6 +227,14 @@ def test_append_and_attention_validate_before_launch():
     for _ in range(4):
         nv.nvkv_ring_push_chunk(d, ring)
     assert _status(nv.nvfp4_kv_append, d, c, ring, kp, vp) == "NVKV_ERR_CAPACITY"
+    assert _status(L.nvfp4_kv_append_spatial_rope, d, c, ring, kp, vp) == "NVKV_ERR_CAPACITY"
+    wide = nv.nvkv_desc_init(1, 2, 8, 91, 1, 1, 3)             # grid_w above 90
+    assert _status(L.nvfp4_kv_append_spatial_rope, wide, c, nv.nvkv_ring_init(wide), kp,
+                   vp) == "NVKV_ERR_UNSUPPORTED"
+    sp = nv.nvkv_desc_init(1, 2, 8, 8, 1, 1, 3)
+    sp.rope_split[0], sp.rope_split[1] = 40, 46
+    assert _status(L.nvfp4_kv_append_spatial_rope, sp, c, nv.nvkv_ring_init(sp), kp,
+                   vp) == "NVKV_ERR_UNSUPPORTED"
     assert _status(nv.chunk_attention_nvfp4kv, d, c, ring, None, op) == "NVKV_ERR_INVALID_ARG"
     assert _status(nv.chunk_attention_bf16kv, d, c, ring, qp, op) == "NVKV_ERR_STATE"
     split = nv.nvkv_desc_init(1, 2, 8, 8, 1, 1, 3)

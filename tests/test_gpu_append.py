@@ -144,3 +144,48 @@ def test_append_extreme_scales_bit_exact(first_scale, later_scale):
             assert np.array_equal(lib.cache.global_scales().cpu().numpy(), ora.s_g)
         _check_new_frames(lib, ora, new)
     assert lib.cache.device_status() == 0
+
+
+ODD60 = kvsynth.Workload("odd60", B=2, H=3, D=128, grid_h=6, grid_w=10, C=2, S=1, W=6, steps=5)
+
+
+@pytest.mark.parametrize("name,count,steps", [("tiny", 1, 6), ("tiny", 4, 6), ("odd60", 4, 5),
+                                              ("stream1p3b", 1, 2), ("stream5b", 2, 2)])
+def test_spatial_rope_append_bit_exact(name, count, steps):
+    """The append of the block-scaled FP4 Q K^T reading (K's h and w pairs
+    rotated in float before quantizing) against the oracle's fp4_qk stream:
+    s_g and every new frame's codes and scales bit for bit, on whole caches
+    and shards (odd ones included) across ring wrap."""
+    import nvfp4_kv_cache_append_b200 as nv
+    from oracle.merge import shard_tokens
+    wl = ODD60 if name == "odd60" else kvsynth.WORKLOADS[name]
+    shards = [nv.KVCache(wl.B, wl.H, wl.grid_h, wl.grid_w, wl.C, wl.S, wl.W, nv.NVKV_KV_NVFP4,
+                         shard_rank=r, shard_count=count) for r in range(count)]
+    ora = OracleStream(wl, seed=7, keep_inputs=False, fp4_qk=True)
+    for step in range(1, steps + 1):
+        x = kvsynth.chunk_qkv(wl, step, 7)
+        new = ora.step(k=x["k"], v=x["v"], q=x["q"])
+        g = to_gpu(x)
+        for c in shards:
+            need = wl.C - min(c.free_frames(b) for b in range(wl.B))
+            if need > 0:
+                c.evict(need)
+            c.append_spatial_rope(g["k"], g["v"])
+        torch.cuda.synchronize()
+        for r, c in enumerate(shards):
+            assert c.device_status() == 0
+            assert np.array_equal(c.global_scales().cpu().numpy(), ora.s_g), (step, r)
+            t0, t1 = shard_tokens(wl.T, count, r)
+            ts, tr = c.Ts, c.Tr
+            for b in range(wl.B):
+                st = c.ring.s[b]
+                slot_of = {st.frame[i]: st.slot[i] for i in range(st.n_resident)}
+                for fid in new[b]:
+                    p = slot_of[fid]
+                    e = ora.frame(b, fid)
+                    rows = slice(p * tr, p * tr + ts)
+                    for w in ("k", "v"):
+                        assert np.array_equal(c.codes(w)[b, :, rows].cpu().numpy(),
+                                              e[w + "_codes"][:, t0:t1]), (step, r, b, fid, w)
+                        assert np.array_equal(c.scales(w)[b, :, rows].cpu().numpy(),
+                                              e[w + "_scales"][:, t0:t1]), (step, r, b, fid, w)
