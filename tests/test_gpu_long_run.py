@@ -1,7 +1,7 @@
 """Long streaming run (1.3B-like shapes, 600 AR steps with ring eviction):
 codes and scales match the oracle at steps 1, 10, 100 and 600, attention at
-step 600 matches on sampled rows, the cache footprint is constant and no
-device memory is allocated per step."""
+steps 100 and 600 matches on sampled rows of every head, the cache
+footprint is constant and no device memory is allocated per step."""
 import numpy as np
 import pytest
 import torch
@@ -20,8 +20,9 @@ def test_long_run_600_steps():
     import nvfp4_kv_cache_append_b200 as nv
     wl = kvsynth.WORKLOADS["long600"]
     C, T = wl.C, wl.T
-    window_steps = set(range(wl.steps - wl.W // C + 1, wl.steps + 1))   # resident at the end
-    oracle_steps = set(CHECK) | window_steps
+    MID = 100
+    window = lambda s: set(range(s - wl.W // C + 1, s + 1))      # steps resident at step s
+    oracle_steps = set(CHECK) | window(wl.steps) | window(MID)
     lib = LibStream(wl, nv.NVKV_KV_NVFP4)
     gen = torch.Generator(device="cuda")
     gen.manual_seed(12345)
@@ -40,6 +41,8 @@ def test_long_run_600_steps():
                  for n in "qkv"}
         out, _ = lib.step(g["q"], g["k"], g["v"], with_lse=False)
         new = ring.step()
+        if step == MID:
+            mid = (out.cpu(), ring.visible(), ring.query_pos0())      # host copy: no device memory
         if step == 1:
             xf = {n: x[n].float().numpy() for n in "kv"}
             s_g = np.array([[oracle.global_scale(oracle.amax(np.ascontiguousarray(xf[n][0, :, h])))
@@ -73,25 +76,28 @@ def test_long_run_600_steps():
     assert torch.cuda.mem_get_info()[0] >= free0 - (64 << 20)
     assert ring.resident() == lib.cache.visible(0)[2]
 
-    # attention at step 600 on sampled rows, from regenerated inputs only
-    q = kept[wl.steps]["q"][0]
+    # attention at steps 100 and 600 on sampled rows of every head, from
+    # regenerated inputs only
     fid_step = lambda fid: (fid // C + 1, fid % C)
-    for h in (0, 5, 11):
-        ks, vs, fpos, tok = [], [], [], []
-        for fid, rank in ring.visible():
-            st, c = fid_step(fid)
-            src = kept[st]
-            for t, (n, lst) in enumerate((("k", ks), ("v", vs))):
-                rows_in = src[n][0, c * T:(c + 1) * T, h].float().numpy()
-                codes, scales = oracle.quantize_rows(rows_in, s_g[t, h])
-                lst.append(oracle.dequant_rows(codes, scales, s_g[t, h]))
-            fpos.append(np.full(T, rank, np.int32))
-            tok.append(np.arange(T, dtype=np.int32))
-        l = np.arange(wl.Lq)
-        qpos = (ring.query_pos0() + l // T).astype(np.int32)
-        rows = sample_rows(wl.Lq, 8, h)
-        ref, _ = oracle.attention_rows(q[:, h], np.concatenate(ks), np.concatenate(vs),
-                                       np.concatenate(fpos), np.concatenate(tok), qpos,
-                                       (l % T).astype(np.int32), rows, wl.grid_w)
-        got = out[0, rows, h].float().cpu().numpy()
-        assert_parity(got, ref, f"step 600 head {h}")
+    for at_step, got_out, visible, qpos0 in ((MID,) + mid, (wl.steps, out, ring.visible(),
+                                                              ring.query_pos0())):
+        q = kept[at_step]["q"][0]
+        for h in range(wl.H):
+            ks, vs, fpos, tok = [], [], [], []
+            for fid, rank in visible:
+                st, c = fid_step(fid)
+                src = kept[st]
+                for t, (n, lst) in enumerate((("k", ks), ("v", vs))):
+                    rows_in = src[n][0, c * T:(c + 1) * T, h].float().numpy()
+                    codes, scales = oracle.quantize_rows(rows_in, s_g[t, h])
+                    lst.append(oracle.dequant_rows(codes, scales, s_g[t, h]))
+                fpos.append(np.full(T, rank, np.int32))
+                tok.append(np.arange(T, dtype=np.int32))
+            l = np.arange(wl.Lq)
+            qpos = (qpos0 + l // T).astype(np.int32)
+            rows = sample_rows(wl.Lq, 12, 31 * at_step + h)
+            ref, _ = oracle.attention_rows(q[:, h], np.concatenate(ks), np.concatenate(vs),
+                                           np.concatenate(fpos), np.concatenate(tok), qpos,
+                                           (l % T).astype(np.int32), rows, wl.grid_w)
+            got = got_out[0, rows, h].float().cpu().numpy()
+            assert_parity(got, ref, f"step {at_step} head {h}")
