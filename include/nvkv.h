@@ -280,6 +280,27 @@ NVKV_API nvkv_status nvfp4_kv_append_spatial_rope(const nvkv_desc *desc, const n
                                                   nvkv_ring *ring, const void *k, const void *v,
                                                   nvkv_stream stream);
 
+/* The query side of the same reading: every row of the chunk's Q quantized
+ * to NVFP4 once per visible key frame.  For the frame at RoPE index f_k
+ * (visible frame j of the stream, in nvkv_ring_visible's order), Q_fk is the
+ * row with its 44-channel frame segment rotated by f_q - f_k (f_q the RoPE
+ * index of the row's own frame) and its h and w segments at the row's (h,
+ * w), all in float as nvfp4_kv_append_spatial_rope rotates K; it is
+ * quantized with the cache's block rule under the row's global scale s_gq =
+ * fl32(p / 2688), p the largest pair magnitude fl32(sqrt(fl32(x^2) +
+ * fl32(y^2))) of the row (which no rotation changes; 1 if not a normal
+ * float).  Then the dot product of the dequantized Q_fk and cached K' rows
+ * equals the rotated q . k of chunk_attention_nvfp4kv up to the two
+ * quantizations.  q: device bf16 [B][Lq][H][128], pre-RoPE.  Outputs, device:
+ * codes [B][H][Lq][S+W][64] (8-byte aligned), scales [B][H][Lq][S+W][8]
+ * (E4M3 codes), s_gq [B][H][Lq] f32; entries j >= the stream's visible
+ * frames are not written.  NVKV_ERR_STATE before the first append;
+ * NVKV_ERR_UNSUPPORTED unless the RoPE split is 44/42/42 and grid_h + grid_w
+ * <= 100. */
+NVKV_API nvkv_status nvkv_fp4qk_quantize_q(const nvkv_desc *desc, const nvkv_ring *ring,
+                                           const void *q, uint8_t *codes, uint8_t *scales,
+                                           float *s_gq, nvkv_stream stream);
+
 /* The bf16-KV twin: same slot logic, the chunk's bf16 K/V copied as is. */
 NVKV_API nvkv_status bf16_kv_append(const nvkv_desc *desc, const nvkv_cache *cache, nvkv_ring *ring,
                            const void *k, const void *v, nvkv_stream stream);

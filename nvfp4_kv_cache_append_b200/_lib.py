@@ -102,6 +102,7 @@ def _load():
         "bf16_kv_append": (i32, [D, C, R, vp, vp, vp]),
         "nvfp4_kv_append_noalloc": (i32, [D, C, R, vp, vp, vp]),
         "nvfp4_kv_append_spatial_rope": (i32, [D, C, R, vp, vp, vp]),
+        "nvkv_fp4qk_quantize_q": (i32, [D, R, vp, vp, vp, vp, vp]),
         "nvfp4_kv_overwrite": (i32, [D, C, R, vp, vp, vp]),
         "bf16_kv_overwrite": (i32, [D, C, R, vp, vp, vp]),
         "nvkv_attention_workspace_bytes": (sz, [D]),
@@ -257,6 +258,11 @@ def nvfp4_kv_append_spatial_rope(desc, cache, ring, k_ptr, v_ptr, stream=0) -> N
     _check(lib.nvfp4_kv_append_spatial_rope(ctypes.byref(desc), ctypes.byref(cache),
                                             ctypes.byref(ring), k_ptr, v_ptr, stream),
            "nvfp4_kv_append_spatial_rope")
+
+
+def nvkv_fp4qk_quantize_q(desc, ring, q_ptr, codes_ptr, scales_ptr, s_gq_ptr, stream=0) -> None:
+    _check(lib.nvkv_fp4qk_quantize_q(ctypes.byref(desc), ctypes.byref(ring), q_ptr, codes_ptr,
+                                     scales_ptr, s_gq_ptr, stream), "nvkv_fp4qk_quantize_q")
 
 
 def bf16_kv_append(desc, cache, ring, k_ptr, v_ptr, stream=0) -> None:

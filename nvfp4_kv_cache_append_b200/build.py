@@ -8,7 +8,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libnvkv.so")
-SOURCES = ["nvkv_host.cpp", "append.cu", "attention.cu", "append_noalloc.cu", "merge.cu", "project.cu"]
+SOURCES = ["nvkv_host.cpp", "append.cu", "attention.cu", "append_noalloc.cu", "merge.cu", "project.cu",
+           "fp4qk.cu"]
 HEADERS = ["nvkv_internal.h", "ptx.cuh", "nvfp4_quant.cuh", os.path.join("..", "..", "include", "nvkv.h")]
 
 NVCC_FLAGS = [

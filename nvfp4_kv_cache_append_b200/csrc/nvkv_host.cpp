@@ -504,6 +504,60 @@ nvkv_status nvfp4_kv_append_spatial_rope(const nvkv_desc *desc, const nvkv_cache
                          nullptr, true);
 }
 
+nvkv_status nvkv_fp4qk_quantize_q(const nvkv_desc *desc, const nvkv_ring *ring, const void *q,
+                                  uint8_t *codes, uint8_t *scales, float *s_gq,
+                                  nvkv_stream stream)
+{
+    nvkv_status st = check_desc(desc);
+    if (st != NVKV_OK) return st;
+    if ((st = check_ring(desc, ring)) != NVKV_OK) return st;
+    if (ring->steps < 1) return NVKV_ERR_STATE;
+    if (!q || !codes || !scales || !s_gq) return NVKV_ERR_INVALID_ARG;
+    if (!aligned16(q) || (reinterpret_cast<uintptr_t>(codes) & 7u) ||
+        (reinterpret_cast<uintptr_t>(s_gq) & 3u))
+        return NVKV_ERR_ALIGNMENT;
+    if (desc->rope_split[0] != 44 || desc->rope_split[1] != 42 || desc->rope_split[2] != 42 ||
+        desc->grid_h + desc->grid_w > nvkv::kQfkMaxSpatial)
+        return NVKV_ERR_UNSUPPORTED;
+    static thread_local nvkv::QfkLaunch a;
+    a = nvkv::QfkLaunch{};
+    a.q = q;
+    a.codes = codes;
+    a.scales = scales;
+    a.s_gq = s_gq;
+    a.B = desc->B;
+    a.H = desc->H;
+    a.T = desc->grid_h * desc->grid_w;
+    a.Lq = desc->C * a.T;
+    a.grid_h = desc->grid_h;
+    a.grid_w = desc->grid_w;
+    a.max_vis = desc->S + desc->W;
+    for (int b = 0; b < desc->B; ++b) {
+        const nvkv_ring_stream &s = ring->s[b];
+        if (s.n_resident < desc->C) return NVKV_ERR_STATE;
+        int n = 0;
+        for (int i = 0; i < s.n_resident; ++i)
+            if (is_visible(s, i)) a.vis_pos[b][n++] = (uint8_t)i;
+        a.n_vis[b] = n;
+        a.q_pos0[b] = s.n_resident - desc->C;
+    }
+    // cos and sin of the fp64 angle pos * base^(-2i/d), each rounded once to float
+    auto cs = [&](int pos, int i, int d) {
+        const double ang = (double)pos * std::pow((double)desc->rope_base, -2.0 * i / (double)d);
+        return make_float2((float)std::cos(ang), (float)std::sin(ang));
+    };
+    for (int dpos = -(nvkv::kQfkMaxChunk - 1); dpos < NVKV_MAX_FRAMES; ++dpos)
+        for (int i = 0; i < 22; ++i)
+            a.fr[(dpos + nvkv::kQfkMaxChunk - 1) * 22 + i] = cs(dpos, i, desc->rope_split[0]);
+    for (int pos = 0; pos < desc->grid_h; ++pos)
+        for (int i = 0; i < 21; ++i) a.sp[pos * 21 + i] = cs(pos, i, desc->rope_split[1]);
+    for (int pos = 0; pos < desc->grid_w; ++pos)
+        for (int i = 0; i < 21; ++i)
+            a.sp[(desc->grid_h + pos) * 21 + i] = cs(pos, i, desc->rope_split[2]);
+    return nvkv::launch_fp4qk_quantize_q(a, (cudaStream_t)stream) == cudaSuccess ? NVKV_OK
+                                                                                : NVKV_ERR_CUDA;
+}
+
 nvkv_status nvfp4_kv_overwrite(const nvkv_desc *desc, const nvkv_cache *cache,
                                const nvkv_ring *ring, const void *k, const void *v,
                                nvkv_stream stream)

@@ -36,6 +36,27 @@ struct SpatialRope {
 };
 cudaError_t launch_nvfp4_append_rope(const AppendLaunch &a, const SpatialRope &r, cudaStream_t s);
 
+// Q of the block-scaled FP4 Q K^T reading, quantized per visible key frame.
+// fr[(dpos + kQfkMaxChunk - 1) * 22 + i]: cos and sin (float) of frame pair i
+// at relative index dpos in [-(kQfkMaxChunk - 1), NVKV_MAX_FRAMES - 1];
+// sp[pos * 21 + i] for h rows pos < grid_h, sp[(grid_h + pos) * 21 + i] for w
+// columns.  Kernel parameter, about 30 KB.
+constexpr int kQfkMaxChunk = NVKV_MAX_CHUNK;
+constexpr int kQfkMaxSpatial = 100;          // grid_h + grid_w
+struct QfkLaunch {
+    const void *q;                           // bf16 [B][Lq][H][128]
+    uint8_t *codes, *scales;                 // [B][H][Lq][max_vis][64], [..][8]
+    float *s_gq;                             // [B][H][Lq]
+    int B, H, Lq, T, grid_h, grid_w, max_vis;
+    int n_vis[NVKV_MAX_BATCH];
+    int q_pos0[NVKV_MAX_BATCH];
+    uint8_t vis_pos[NVKV_MAX_BATCH][NVKV_MAX_FRAMES];   // RoPE frame index of visible frame j
+    float2 fr[(kQfkMaxChunk - 1 + NVKV_MAX_FRAMES) * 22];
+    float2 sp[kQfkMaxSpatial * 21];
+};
+static_assert(sizeof(QfkLaunch) <= 32764, "kernel parameter space");
+cudaError_t launch_fp4qk_quantize_q(const QfkLaunch &a, cudaStream_t s);
+
 // Tokens per frame of the cache a desc describes (the shard's share of each
 // frame) and the index of its first token within the frame.
 inline int shard_tokens(const nvkv_desc *d)

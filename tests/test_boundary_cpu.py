@@ -231,6 +231,15 @@ def test_append_and_attention_validate_before_launch():
     wide = nv.nvkv_desc_init(1, 2, 8, 91, 1, 1, 3)             # grid_w above 90
     assert _status(L.nvfp4_kv_append_spatial_rope, wide, c, nv.nvkv_ring_init(wide), kp,
                    vp) == "NVKV_ERR_UNSUPPORTED"
+    fake = 1 << 20
+    empty = nv.nvkv_ring_init(d)
+    assert _status(L.nvkv_fp4qk_quantize_q, d, empty, kp, fake, fake, fake) == "NVKV_ERR_STATE"
+    assert _status(L.nvkv_fp4qk_quantize_q, d, ring, None, fake, fake, fake) == "NVKV_ERR_INVALID_ARG"
+    assert _status(L.nvkv_fp4qk_quantize_q, d, ring, kp, fake + 4, fake, fake) == "NVKV_ERR_ALIGNMENT"
+    big = nv.nvkv_desc_init(1, 2, 50, 51, 1, 1, 3)               # grid_h + grid_w above 100
+    rb = nv.nvkv_ring_init(big)
+    nv.nvkv_ring_push_chunk(big, rb)
+    assert _status(L.nvkv_fp4qk_quantize_q, big, rb, kp, fake, fake, fake) == "NVKV_ERR_UNSUPPORTED"
     sp = nv.nvkv_desc_init(1, 2, 8, 8, 1, 1, 3)
     sp.rope_split[0], sp.rope_split[1] = 40, 46
     assert _status(L.nvfp4_kv_append_spatial_rope, sp, c, nv.nvkv_ring_init(sp), kp,
