@@ -301,6 +301,27 @@ NVKV_API nvkv_status nvkv_fp4qk_quantize_q(const nvkv_desc *desc, const nvkv_rin
                                            const void *q, uint8_t *codes, uint8_t *scales,
                                            float *s_gq, nvkv_stream stream);
 
+/* The contraction of the same reading on the block-scaled tensor cores
+ * (tcgen05.mma kind::mxf4nvf4, E2M1 operands, UE4M3 block scales per 16):
+ * the logit of every query row against every visible cached key,
+ *   out = (sum over blocks of sA sB sum of code products) * s_gq * s_g(K),
+ * i.e. the dot product of the dequantized Q_fk and K' rows (without the
+ * 1/sqrt(128) of the softmax).  q_codes, q_scales, s_gq: the outputs of
+ * nvkv_fp4qk_quantize_q for this step; the cache must have been filled by
+ * nvfp4_kv_append_spatial_rope.  out: device f32 [B][H][Lq][S+W][Ts], entry
+ * (row, j, i) the logit against token i of the stream's visible frame j
+ * (entries of frames past the visible ones are not written).  It writes the
+ * whole logit matrix (Lq x visible keys per head), so it suits small shapes;
+ * a fused attention would keep each tile in TMEM.  NVKV_ERR_STATE for a bf16
+ * cache or before the first append; NVKV_ERR_ALIGNMENT unless q_codes and
+ * k_data are 16-byte, the scale arrays 8-byte and s_gq and out 4-byte
+ * aligned; the status word receives NVKV_ERR_TIMEOUT if an MMA wait runs
+ * out. */
+NVKV_API nvkv_status nvkv_fp4qk_scores(const nvkv_desc *desc, const nvkv_cache *cache,
+                                       const nvkv_ring *ring, const uint8_t *q_codes,
+                                       const uint8_t *q_scales, const float *s_gq, float *out,
+                                       nvkv_stream stream);
+
 /* The bf16-KV twin: same slot logic, the chunk's bf16 K/V copied as is. */
 NVKV_API nvkv_status bf16_kv_append(const nvkv_desc *desc, const nvkv_cache *cache, nvkv_ring *ring,
                            const void *k, const void *v, nvkv_stream stream);

@@ -103,6 +103,7 @@ def _load():
         "nvfp4_kv_append_noalloc": (i32, [D, C, R, vp, vp, vp]),
         "nvfp4_kv_append_spatial_rope": (i32, [D, C, R, vp, vp, vp]),
         "nvkv_fp4qk_quantize_q": (i32, [D, R, vp, vp, vp, vp, vp]),
+        "nvkv_fp4qk_scores": (i32, [D, C, R, vp, vp, vp, vp, vp]),
         "nvfp4_kv_overwrite": (i32, [D, C, R, vp, vp, vp]),
         "bf16_kv_overwrite": (i32, [D, C, R, vp, vp, vp]),
         "nvkv_attention_workspace_bytes": (sz, [D]),
@@ -263,6 +264,13 @@ def nvfp4_kv_append_spatial_rope(desc, cache, ring, k_ptr, v_ptr, stream=0) -> N
 def nvkv_fp4qk_quantize_q(desc, ring, q_ptr, codes_ptr, scales_ptr, s_gq_ptr, stream=0) -> None:
     _check(lib.nvkv_fp4qk_quantize_q(ctypes.byref(desc), ctypes.byref(ring), q_ptr, codes_ptr,
                                      scales_ptr, s_gq_ptr, stream), "nvkv_fp4qk_quantize_q")
+
+
+def nvkv_fp4qk_scores(desc, cache, ring, q_codes_ptr, q_scales_ptr, s_gq_ptr, out_ptr,
+                      stream=0) -> None:
+    _check(lib.nvkv_fp4qk_scores(ctypes.byref(desc), ctypes.byref(cache), ctypes.byref(ring),
+                                 q_codes_ptr, q_scales_ptr, s_gq_ptr, out_ptr, stream),
+           "nvkv_fp4qk_scores")
 
 
 def bf16_kv_append(desc, cache, ring, k_ptr, v_ptr, stream=0) -> None:

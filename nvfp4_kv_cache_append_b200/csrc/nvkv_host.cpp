@@ -558,6 +558,49 @@ nvkv_status nvkv_fp4qk_quantize_q(const nvkv_desc *desc, const nvkv_ring *ring, 
                                                                                 : NVKV_ERR_CUDA;
 }
 
+nvkv_status nvkv_fp4qk_scores(const nvkv_desc *desc, const nvkv_cache *cache,
+                              const nvkv_ring *ring, const uint8_t *q_codes,
+                              const uint8_t *q_scales, const float *s_gq, float *out,
+                              nvkv_stream stream)
+{
+    nvkv_status st = check_desc(desc);
+    if (st != NVKV_OK) return st;
+    if (desc->kv_dtype != NVKV_KV_NVFP4) return NVKV_ERR_STATE;
+    if ((st = check_ring(desc, ring)) != NVKV_OK) return st;
+    if (ring->steps < 1) return NVKV_ERR_STATE;
+    if (!cache || !cache->k_data || !cache->k_scales || !cache->s_g || !cache->status || !q_codes ||
+        !q_scales || !s_gq || !out)
+        return NVKV_ERR_INVALID_ARG;
+    if (!aligned16(q_codes) || (reinterpret_cast<uintptr_t>(q_scales) & 7u) ||
+        !aligned16(cache->k_data) || (reinterpret_cast<uintptr_t>(cache->k_scales) & 7u) ||
+        (reinterpret_cast<uintptr_t>(s_gq) & 3u) || (reinterpret_cast<uintptr_t>(out) & 3u))
+        return NVKV_ERR_ALIGNMENT;
+    nvkv::ScoreLaunch a{};
+    a.q_codes = q_codes;
+    a.q_scales = q_scales;
+    a.s_gq = s_gq;
+    a.k_codes = static_cast<const uint8_t *>(cache->k_data);
+    a.k_scales = static_cast<const uint8_t *>(cache->k_scales);
+    a.s_gk = cache->s_g;
+    a.out = out;
+    a.status = cache->status;
+    a.B = desc->B;
+    a.H = desc->H;
+    a.Lq = desc->C * desc->grid_h * desc->grid_w;
+    a.R = (int)rows_per_head(desc);
+    a.Tk = nvkv::shard_tokens(desc);
+    a.Tr = nvkv::slot_rows(desc);
+    a.max_vis = desc->S + desc->W;
+    for (int b = 0; b < desc->B; ++b) {
+        const nvkv_ring_stream &s = ring->s[b];
+        int n = 0;
+        for (int i = 0; i < s.n_resident; ++i)
+            if (is_visible(s, i)) a.vis_slot[b][n++] = (uint16_t)s.slot[i];
+        a.n_vis[b] = n;
+    }
+    return nvkv::launch_fp4qk_scores(a, (cudaStream_t)stream) == cudaSuccess ? NVKV_OK : NVKV_ERR_CUDA;
+}
+
 nvkv_status nvfp4_kv_overwrite(const nvkv_desc *desc, const nvkv_cache *cache,
                                const nvkv_ring *ring, const void *k, const void *v,
                                nvkv_stream stream)

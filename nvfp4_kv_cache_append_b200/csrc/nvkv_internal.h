@@ -55,6 +55,22 @@ struct QfkLaunch {
     float2 sp[kQfkMaxSpatial * 21];
 };
 static_assert(sizeof(QfkLaunch) <= 32764, "kernel parameter space");
+
+// The FP4 contraction of the same reading: logits of every query row against
+// every visible key, from the quantized Q_fk (nvkv_fp4qk_quantize_q) and the
+// cached K' (nvfp4_kv_append_spatial_rope), on block-scaled tensor-core MMAs.
+struct ScoreLaunch {
+    const uint8_t *q_codes, *q_scales;      // [B][H][Lq][max_vis][64], [..][8]
+    const float *s_gq;                      // [B][H][Lq]
+    const uint8_t *k_codes, *k_scales;      // cache planes [B][H][R][64], [..][8]
+    const float *s_gk;                      // [B][H] (K's global scales)
+    float *out;                             // [B][H][Lq][max_vis][Tk]
+    int32_t *status;
+    int B, H, Lq, R, Tk, Tr, max_vis;
+    int n_vis[NVKV_MAX_BATCH];
+    uint16_t vis_slot[NVKV_MAX_BATCH][NVKV_MAX_FRAMES];
+};
+cudaError_t launch_fp4qk_scores(const ScoreLaunch &a, cudaStream_t s);
 cudaError_t launch_fp4qk_quantize_q(const QfkLaunch &a, cudaStream_t s);
 
 // Tokens per frame of the cache a desc describes (the shard's share of each
