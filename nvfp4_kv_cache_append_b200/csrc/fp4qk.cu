@@ -237,11 +237,15 @@ __global__ void __launch_bounds__(128) k_fp4qk_scores(const __grid_constant__ Sc
         }
         const int never = 0;
         const bool ok = ptx::mbar_wait(&bar, phase, &never, 2000000000ull);
-        phase ^= 1;
         if (!__syncthreads_and(ok)) {
-            if (t == 0) atomicCAS(a.status, 0, (int)NVKV_ERR_TIMEOUT);
+            // give the MMAs one more bounded wait before TMEM is released
+            if (t == 0) {
+                atomicCAS(a.status, 0, (int)NVKV_ERR_TIMEOUT);
+                ptx::mbar_wait(&bar, phase, &never, 2000000000ull);
+            }
             break;
         }
+        phase ^= 1;
         ptx::tc_fence_after();
         // lane t of the accumulator is query row row0 + t; column c key key0 + c
         const uint32_t tq = tD + ((uint32_t)(warp * 32) << 16);

@@ -236,6 +236,16 @@ def test_append_and_attention_validate_before_launch():
     assert _status(L.nvkv_fp4qk_quantize_q, d, empty, kp, fake, fake, fake) == "NVKV_ERR_STATE"
     assert _status(L.nvkv_fp4qk_quantize_q, d, ring, None, fake, fake, fake) == "NVKV_ERR_INVALID_ARG"
     assert _status(L.nvkv_fp4qk_quantize_q, d, ring, kp, fake + 4, fake, fake) == "NVKV_ERR_ALIGNMENT"
+    sc = L.nvkv_fp4qk_scores
+    assert _status(sc, d, c, empty, fake, fake, fake, fake) == "NVKV_ERR_STATE"       # no append yet
+    assert _status(sc, d, c, ring, None, fake, fake, fake) == "NVKV_ERR_INVALID_ARG"
+    assert _status(sc, d, c, ring, fake + 8, fake, fake, fake) == "NVKV_ERR_ALIGNMENT"
+    assert _status(sc, d, c, ring, fake, fake + 4, fake, fake) == "NVKV_ERR_ALIGNMENT"
+    assert _status(sc, d, c, ring, fake, fake, fake, fake + 2) == "NVKV_ERR_ALIGNMENT"
+    tw = nv.nvkv_desc_init(1, 2, 8, 8, 1, 1, 3, nv.NVKV_KV_BF16)
+    rt = nv.nvkv_ring_init(tw)
+    nv.nvkv_ring_push_chunk(tw, rt)
+    assert _status(sc, tw, c, rt, fake, fake, fake, fake) == "NVKV_ERR_STATE"         # bf16 cache
     big = nv.nvkv_desc_init(1, 2, 50, 51, 1, 1, 3)               # grid_h + grid_w above 100
     rb = nv.nvkv_ring_init(big)
     nv.nvkv_ring_push_chunk(big, rb)
